@@ -1,0 +1,24 @@
+"""CPU oracle (float64) for exact split decode attention.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the library.  It shares no
+code with the CUDA library.  See ``attention.py`` for the definitions and the
+passages they follow.
+"""
+from .attention import (  # noqa: F401
+    Partial,
+    attention_one,
+    attention_one_bf16_cache,
+    bf16_to_f64,
+    bifurcated_attention,
+    chunk_partial,
+    decode_attention,
+    energy,
+    finalize,
+    merge,
+    merge_tree,
+    online_softmax,
+    sequence_block,
+    split_attention,
+    to_f64,
+)

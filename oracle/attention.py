@@ -1,0 +1,292 @@
+"""CPU oracle for exact split decode attention.
+
+TEST INFRASTRUCTURE.  This module is the correctness reference for the CUDA
+library.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` may import or call it; the library never does, and it shares no
+code with the library (it reads the same host input bytes, nothing else).
+
+Everything is computed in float64 on the exact input values (bf16 and float32
+inputs widen to float64 without rounding).
+
+Sources (the web pages this method is taken from):
+
+* [AttnAccel] "Attention acceleration" (compassingai.com, concept page
+  attention-acceleration), section "Technical principles": part 1 "Self-attention
+  recap" gives S = Q K^T / sqrt(d_k), P = softmax(S), O = P V; part 2.1
+  "Tiling and online softmax" gives m(x) = max_j x_j, l(x) = sum_j exp(x_j - m(x))
+  and the block update of m, l and O.
+* [TreeAttn] Tree Attention article (m.srwj168.com.cn, keji312/12691), section
+  "The energy view of attention": attention is the gradient, at zeta = 0, of a
+  scalar energy F(K, Q, V, zeta); logsumexp and max are associative, so the
+  per-device pieces can be combined in any order (tree all-reduce).
+* [Bifurcated] Bifurcated attention summary (briefgpt.xyz, 2403.08845), TL;DR:
+  decode attention over a shared prefilled context plus per-sample decoded
+  tokens is split into two GEMMs and stays exact.
+* [StarAttn] Star Attention article (tiaojiaomugou.com, 242533), "Phase 2: query
+  encoding and token generation": each host attends over its local cache and the
+  query host combines the softmax statistics into global attention.
+
+Readings taken where the pages are silent or garbled (each also listed in the
+design notes):
+
+1. The decode energy formula did not survive extraction.  It is read as
+   F(zeta) = log sum_t exp(s * q.k_t + zeta.v_t); then dF/dzeta at 0 = output.
+2. lse is the natural logarithm of sum_t exp(s * q.k_t) (scaled scores).
+3. The online-softmax output update of [AttnAccel] 2.1 is printed in the
+   normalised form with an undefined "block_result"; it is read as
+   sum_{j in block} exp(x_j - m_new) v_j.  The split path keeps O unnormalised
+   (the partial (m, l, o)), which is algebraically the same.
+4. An empty sequence gives out = 0 and lse = -inf.
+5. GQA: query head h reads KV head h // (Hq / Hkv) (consecutive groups).
+6. The bifurcated result for sample n is plain attention over the concatenation
+   [prefix ; suffix_n]; no mask (the query is the last position).
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+Partial = Tuple[float, float, np.ndarray]  # (m, l, o): running max, sum of exponentials, unnormalised output
+
+# Rows of K and V widened to float64 at a time when a cache is decoded in pieces
+# (memory only: every score and every sum term is the same as with one piece).
+ROWS_PER_PIECE = 1 << 20
+
+
+# ------------------------------------------------------------------------------------------
+# Input decoding
+# ------------------------------------------------------------------------------------------
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) to float64: the bf16 value is the float32 whose
+    upper 16 bits are the pattern and whose lower 16 bits are zero (exact)."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return bf16_to_f64(a)
+    if dtype == "f32":
+        return np.asarray(a, dtype=np.float32).astype(np.float64)
+    if dtype == "f64":
+        return np.asarray(a, dtype=np.float64)
+    raise ValueError(dtype)
+
+
+def sequence_block(flat: np.ndarray, seqlens: Sequence[int], b: int, n_kv_heads: int, head_dim: int) -> np.ndarray:
+    """View of sequence b's [Hkv][S_b][D] block in a cache packed sequence after sequence."""
+    start = int(sum(int(s) for s in seqlens[:b])) * n_kv_heads * head_dim
+    S = int(seqlens[b])
+    return flat[start : start + n_kv_heads * S * head_dim].reshape(n_kv_heads, S, head_dim)
+
+
+# ------------------------------------------------------------------------------------------
+# The definition ([AttnAccel] part 1, one decode query)
+# ------------------------------------------------------------------------------------------
+
+
+def attention_one(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> Tuple[np.ndarray, float]:
+    """softmax(scale * K q) V and its log-sum-exp, two passes, float64.
+
+    q: [D]; K, V: [S][D] float64.  Pass 1 forms every score x_t = scale * q.k_t
+    and their maximum m; pass 2 forms l = sum_t exp(x_t - m) and
+    sum_t exp(x_t - m) v_t.  Returns (out = that sum / l, lse = m + ln l).
+    """
+    S, D = K.shape
+    if S == 0:
+        return np.zeros(D), -math.inf
+    x = scale * (K @ q)
+    m = float(np.max(x))
+    e = np.exp(x - m)
+    l = float(np.sum(e))
+    out = (e @ V) / l
+    return out, m + math.log(l)
+
+
+def attention_one_bf16_cache(q: np.ndarray, Kbits: np.ndarray, Vbits: np.ndarray, scale: float,
+                             dtype: str = "bf16") -> Tuple[np.ndarray, float]:
+    """attention_one for a long cache kept in its storage format ([S][D] bf16 bits or float32).
+
+    The cache is widened to float64 ROWS_PER_PIECE rows at a time; pass 1 still
+    forms every score before pass 2 starts, so the arithmetic is the definition's.
+    """
+    S = Kbits.shape[0]
+    D = q.shape[0]
+    if S == 0:
+        return np.zeros(D), -math.inf
+    x = np.empty(S)
+    for r0 in range(0, S, ROWS_PER_PIECE):
+        r1 = min(S, r0 + ROWS_PER_PIECE)
+        x[r0:r1] = scale * (to_f64(Kbits[r0:r1], dtype) @ q)
+    m = float(np.max(x))
+    e = np.exp(x - m)
+    l = float(np.sum(e))
+    acc = np.zeros(D)
+    for r0 in range(0, S, ROWS_PER_PIECE):
+        r1 = min(S, r0 + ROWS_PER_PIECE)
+        acc += e[r0:r1] @ to_f64(Vbits[r0:r1], dtype)
+    return acc / l, m + math.log(l)
+
+
+def decode_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_q_heads: int, n_kv_heads: int,
+                     head_dim: int, scale: float, dtype: str = "bf16",
+                     pairs: Optional[Iterable[Tuple[int, int]]] = None):
+    """Decode attention for a batch with a packed, ragged KV cache.
+
+    q: [B][Hq][D] (storage format); k_cache, v_cache: flat arrays, sequence b's
+    block is [Hkv][S_b][D], blocks back to back.  Query head h of sequence b
+    attends over KV head h // (Hq / Hkv) of sequence b (reading 5).
+
+    Returns (out [B][Hq][D] float64, lse [B][Hq] float64).  With `pairs`, only
+    those (b, h) entries are computed; the rest are NaN.
+    """
+    B = len(seqlens)
+    Hq, Hkv, D = n_q_heads, n_kv_heads, head_dim
+    if Hq % Hkv != 0:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    G = Hq // Hkv
+    qf = to_f64(np.asarray(q).reshape(B, Hq, D), dtype)
+    out = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    todo = sorted(set(pairs)) if pairs is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b in sorted({p[0] for p in todo}):
+        Kb = sequence_block(k_cache, seqlens, b, Hkv, D)
+        Vb = sequence_block(v_cache, seqlens, b, Hkv, D)
+        for g in sorted({h // G for (bb, h) in todo if bb == b}):
+            heads = [h for (bb, h) in todo if bb == b and h // G == g]
+            for h in heads:
+                out[b, h], lse[b, h] = attention_one_bf16_cache(qf[b, h], Kb[g], Vb[g], scale, dtype)
+    return out, lse
+
+
+# ------------------------------------------------------------------------------------------
+# The method's steps: chunk partials and their merge
+# ------------------------------------------------------------------------------------------
+
+
+def chunk_partial(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> Partial:
+    """Softmax statistics of one chunk of the cache ([StarAttn] phase 2; [AttnAccel] 2.1).
+
+    m = max_t x_t, l = sum_t exp(x_t - m), o = sum_t exp(x_t - m) v_t (o is not
+    divided by l).  An empty chunk gives (-inf, 0, 0).
+    """
+    D = q.shape[0]
+    if K.shape[0] == 0:
+        return -math.inf, 0.0, np.zeros(D)
+    x = scale * (K @ q)
+    m = float(np.max(x))
+    e = np.exp(x - m)
+    return m, float(np.sum(e)), e @ V
+
+
+def merge(a: Partial, b: Partial) -> Partial:
+    """Combine the statistics of two disjoint chunks ([TreeAttn]: max and logsumexp are associative).
+
+    m = max(m_a, m_b); each side is rescaled by exp(m_side - m) before l and o
+    are added, as in the l_new update of [AttnAccel] 2.1.
+    """
+    ma, la, oa = a
+    mb, lb, ob = b
+    if ma == -math.inf and mb == -math.inf:
+        return -math.inf, 0.0, np.zeros_like(oa)
+    m = max(ma, mb)
+    ca = math.exp(ma - m) if ma != -math.inf else 0.0
+    cb = math.exp(mb - m) if mb != -math.inf else 0.0
+    return m, la * ca + lb * cb, oa * ca + ob * cb
+
+
+def finalize(p: Partial) -> Tuple[np.ndarray, float]:
+    """out = o / l and lse = m + ln l; (-inf, 0, 0) gives (0, -inf) (reading 4)."""
+    m, l, o = p
+    if l == 0.0:
+        return np.zeros_like(o), -math.inf
+    return o / l, m + math.log(l)
+
+
+def merge_tree(parts: List[Partial]) -> Partial:
+    """Merge partials pairwise, level by level: depth ceil(log2 n) ([TreeAttn] tree all-reduce)."""
+    if not parts:
+        raise ValueError("no partials")
+    level = list(parts)
+    while len(level) > 1:
+        nxt = [merge(level[i], level[i + 1]) for i in range(0, len(level) - 1, 2)]
+        if len(level) % 2:
+            nxt.append(level[-1])
+        level = nxt
+    return level[0]
+
+
+def split_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float,
+                    bounds: Sequence[int]) -> Tuple[np.ndarray, float]:
+    """Attention computed chunk by chunk: chunk c covers rows [bounds[c], bounds[c+1])."""
+    parts = [chunk_partial(q, K[t0:t1], V[t0:t1], scale) for t0, t1 in zip(bounds[:-1], bounds[1:])]
+    return finalize(merge_tree(parts))
+
+
+def online_softmax(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float, block: int) -> Tuple[np.ndarray, float]:
+    """[AttnAccel] 2.1 as printed: blocks of `block` keys, normalised running output.
+
+    m_new = max(m_old, m_block); l_new = l_old exp(m_old - m_new) + sum_block exp(x - m_new);
+    O_new = (O_old l_old exp(m_old - m_new) + sum_block exp(x - m_new) v) / l_new.
+    """
+    S, D = K.shape
+    m, l, O = -math.inf, 0.0, np.zeros(D)
+    for t0 in range(0, S, block):
+        x = scale * (K[t0 : t0 + block] @ q)
+        m_new = max(m, float(np.max(x)))
+        carry = math.exp(m - m_new) if m != -math.inf else 0.0
+        e = np.exp(x - m_new)
+        l_new = l * carry + float(np.sum(e))
+        O = (O * l * carry + e @ V[t0 : t0 + block]) / l_new
+        m, l = m_new, l_new
+    if l == 0.0:
+        return np.zeros(D), -math.inf
+    return O, m + math.log(l)
+
+
+def energy(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float, zeta: np.ndarray) -> float:
+    """F(zeta) = log sum_t exp(scale * q.k_t + zeta.v_t)  ([TreeAttn], reading 1)."""
+    z = scale * (K @ q) + V @ zeta
+    zm = float(np.max(z))
+    return zm + math.log(float(np.sum(np.exp(z - zm))))
+
+
+# ------------------------------------------------------------------------------------------
+# Bifurcated (shared-prefix) decode
+# ------------------------------------------------------------------------------------------
+
+
+def bifurcated_attention(q, k_prefix, v_prefix, prefix_len: int, k_suffix, v_suffix,
+                         suffix_lens: Sequence[int], n_q_heads: int, n_kv_heads: int, head_dim: int,
+                         scale: float, dtype: str = "bf16",
+                         pairs: Optional[Iterable[Tuple[int, int]]] = None):
+    """Sample n, query head h attends over [prefix ; suffix_n] of KV head h // G (reading 6).
+
+    q: [N][Hq][D]; k_prefix, v_prefix: [Hkv][P][D]; k_suffix, v_suffix: packed
+    per sample ([Hkv][S_n][D] blocks back to back).  Returns (out, lse) as
+    decode_attention does.
+    """
+    N = len(suffix_lens)
+    Hq, Hkv, D, P = n_q_heads, n_kv_heads, head_dim, prefix_len
+    G = Hq // Hkv
+    qf = to_f64(np.asarray(q).reshape(N, Hq, D), dtype)
+    Kp = to_f64(np.asarray(k_prefix).reshape(Hkv, P, D), dtype)
+    Vp = to_f64(np.asarray(v_prefix).reshape(Hkv, P, D), dtype)
+    out = np.full((N, Hq, D), np.nan)
+    lse = np.full((N, Hq), np.nan)
+    todo = sorted(set(pairs)) if pairs is not None else [(n, h) for n in range(N) for h in range(Hq)]
+    for n in sorted({p[0] for p in todo}):
+        Ks = to_f64(sequence_block(k_suffix, suffix_lens, n, Hkv, D), dtype)
+        Vs = to_f64(sequence_block(v_suffix, suffix_lens, n, Hkv, D), dtype)
+        for (nn, h) in todo:
+            if nn != n:
+                continue
+            g = h // G
+            K = np.concatenate([Kp[g], Ks[g]], axis=0)
+            V = np.concatenate([Vp[g], Vs[g]], axis=0)
+            out[n, h], lse[n, h] = attention_one(qf[n, h], K, V, scale)
+    return out, lse
