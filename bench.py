@@ -1,0 +1,383 @@
+"""Benchmark: exact split decode attention on B200.
+
+One step = one decode step of the whole hot path (split-KV chunk statistics, their
+log-depth merge and the final normalisation: one fused kernel launch) over the
+long-context workload: batch 1, 32 query heads, 8 KV heads, head_dim 128, KV length
+1,048,576, bf16 K/V ~ N(0,1) with 0.1% of keys scaled x4.  Inputs are synthetic and
+seeded (4.3 GB of K/V, larger than the 126 MB L2, so no flush between steps).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+Prints one JSON line (rank 0).  Under torchrun with N > 1 every rank runs its own
+replica of the workload (no data-path collective: the path does not shard), the
+timed region is bracketed by a barrier and synchronisation, and the time is the max
+over ranks.  `--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode-attn KV GB/s & % of B200 HBM peak at 1M ctx; µs/step, KV tokens/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["exact_long_context_split_b200/csrc/split_kv.cuh", "exact_long_context_split_b200/csrc/ptx.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kv_traffic.json")
+
+
+# ----------------------------------------------------------------------------------------------
+# Host-side pieces shared by every rank (and covered by CPU tests)
+# ----------------------------------------------------------------------------------------------
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """The largest value over all ranks (every rank takes this collective step)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_per_launch(spec) -> object:
+    """DRAM bytes of one launch from the committed ncu summary, scaled to this workload's KV
+    bytes; None when the kernel sources changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            d = json.load(fh)
+    except Exception:
+        return None
+    if d.get("kernel_hash") != kernel_hash():
+        return None
+    return int(round(d["dram_bytes_per_kv_byte"] * spec.kv_bytes))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra) -> dict:
+    rec = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": n_gpus,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype,
+        "data": "synthetic",
+        "config": {
+            "workload": spec.name,
+            "batch": spec.batch,
+            "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
+            "n_q_heads": spec.n_q_heads,
+            "n_kv_heads": spec.n_kv_heads,
+            "head_dim": spec.head_dim,
+            "kv_bytes_per_step": spec.kv_bytes,
+            "parallelism": f"replicas{n_gpus}",
+            "l2": "no flush: each step reads %.2f GB of K/V, more than the 126 MB L2" % (spec.kv_bytes / 1e9),
+        },
+    }
+    rec.update(extra)
+    return rec
+
+
+def oracle_sample_seconds(spec, h_kv: int, q_heads, n_tokens: int = 0) -> float:
+    """Time the CPU oracle on the given query heads of KV head h_kv of sequence 0, over its first
+    n_tokens tokens (0 = all).  Inputs are generated for that head only (the same bytes as the
+    full workload's); only the oracle is timed."""
+    import oracle
+
+    S, D, Hq = spec.seqlens[0], spec.head_dim, spec.n_q_heads
+    n = S * D
+    k = synth.normal_bf16(spec.seed, synth.TID_K, n, start=h_kv * n)
+    v = synth.normal_bf16(spec.seed, synth.TID_V, n, start=h_kv * n)
+    if spec.spike_frac > 0:
+        synth.spike_rows_bf16(k.reshape(S, D), spec.seed, h_kv, spec.n_spikes(S), spec.spike_factor)
+    q = synth.normal_bf16(spec.seed, synth.TID_Q, Hq * D).reshape(Hq, D)
+    T = n_tokens or S
+    K, V = k.reshape(S, D)[:T], v.reshape(S, D)[:T]
+    t0 = time.perf_counter()
+    for h in q_heads:
+        oracle.attention_one_bf16_cache(oracle.bf16_to_f64(q[h]), K, V, spec.scale)
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return 1
+
+
+# ----------------------------------------------------------------------------------------------
+# Reference arm: the CPU oracle
+# ----------------------------------------------------------------------------------------------
+
+
+REF_SLICE = 8  # the reference arm's per-step sample covers 1/REF_SLICE of the sequence
+
+
+def run_reference(args, spec) -> None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    G = spec.n_q_heads // spec.n_kv_heads
+    rows = spec.batch * spec.n_q_heads
+    T = spec.seqlens[0] // REF_SLICE
+    for _ in range(args.warmup):
+        oracle_sample_seconds(spec, 0, [0], T)
+    times = [oracle_sample_seconds(spec, i % spec.n_kv_heads, [(i % spec.n_kv_heads) * G], T) for i in range(args.steps)]
+    step_s = statistics.mean(times) * REF_SLICE * rows
+    value = spec.kv_bytes / step_s / 1e9
+    cores = blas_threads()
+    sample = (f"each step: one (sequence, query head) row over the first {T} of {spec.seqlens[0]} tokens "
+              f"(KV head cycling 0..{spec.n_kv_heads - 1}); step time = mean sample time x {REF_SLICE} x {rows} rows")
+    rec = make_record(value=value, n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
+                      spec=spec, dtype="f64", extra={
+                          "impl": "reference",
+                          "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                          "gpu_launches": 0,
+                      })
+    print(json.dumps(rec), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# The CUDA path
+# ----------------------------------------------------------------------------------------------
+
+
+def run_gpu(args, spec) -> None:
+    import torch
+
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    import exact_long_context_split_b200 as ta
+
+    B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+    seqlens = [int(s) for s in spec.seqlens]
+    inp = synth.make_decode_inputs(spec)
+    host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
+            for n in ("q", "k", "v")}
+    dev = {n: t.cuda() for n, t in host.items()}
+    out = torch.empty(B, Hq, D, device="cuda")
+    lse = torch.empty(B, Hq, device="cuda")
+    ws = torch.empty(ta.tree_attn_workspace_size(seqlens, Hq, Hkv, D), dtype=torch.uint8, device="cuda")
+    ta.tree_attn_workspace_init(ws)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ta.tree_attn_decode_ex("bf16", dev["q"], dev["k"], dev["v"], seqlens, Hq, Hkv, D, spec.scale, out, lse,
+                               None, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ta.tree_attn_check(ws) == ta.TA_OK
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    status = ta.tree_attn_check(ws)
+    if status != ta.TA_OK:
+        raise RuntimeError(ta.tree_attn_status_string(status))
+    elapsed_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
+    kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    ms_per_step = elapsed_ms / args.steps
+    value = world * spec.kv_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # End to end through the public API: pinned host -> device copies of q, K, V, the call, and
+    # the device -> host read of out and lse, every step.
+    e2e_steps = max(1, min(args.steps, 5))
+    out_h = torch.empty(B, Hq, D).pin_memory()
+    lse_h = torch.empty(B, Hq).pin_memory()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for n in ("q", "k", "v"):
+            dev[n].copy_(host[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+
+    peak, peak_kind = measured_peaks()
+    achieved = spec.kv_bytes / (kernel_ms * 1e-3) / 1e9
+    extra = {
+        "ms_per_step": ms_per_step,
+        "us_per_step": ms_per_step * 1e3,
+        "kv_tokens_per_s": world * spec.tokens * args.steps / (elapsed_ms * 1e-3),
+        "hbm_frac_of_" + peak_kind: value / world / peak,
+        "e2e": {"value": world * spec.kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind, "kernel": "split_kv_decode_kernel<bf16,128,4>",
+                     "traffic": traffic_per_launch(spec)},
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        G = Hq // Hkv
+        sec = oracle_sample_seconds(spec, 0, list(range(G)))
+        rows = B * Hq
+        cpu_val = spec.kv_bytes / (sec / G * rows) / 1e9
+        extra["cpu_baseline"] = {"value": cpu_val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"the {G} query heads of KV head 0 over all {spec.seqlens[0]} tokens took "
+                                           f"{sec:.2f} s; step time = that / {G} x {rows} rows"}
+    rec = make_record(value=value, n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=ms_per_step,
+                      spec=spec, dtype="bf16", extra=extra)
+    if rank == 0:
+        print(json.dumps(rec), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="long_1m", choices=sorted(synth.decode_configs()))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    spec = synth.decode_configs()[args.workload]
+    if args.impl == "reference":
+        run_reference(args, spec)
+    else:
+        run_gpu(args, spec)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,605 @@
+// Split-KV decode attention: one persistent CTA per SM streams an equal share of
+// the whole job's KV tiles through a 4-stage shared-memory ring (bulk copies on
+// the TMA engine), computes exp2-domain online-softmax statistics (m, l, o) for
+// the G query heads that share each KV head, and merges the statistics of the
+// CTAs that shared a (sequence, KV head) in a fixed pairwise tree.
+//
+// Method: "Attention acceleration" concept page (compassingai.com), Technical
+// principles part 1 (S = QK^T/sqrt(d_k), P = softmax(S), O = PV) and part 2.1
+// (online softmax: m_new = max(m_old, m_block), l_new = l_old e^{m_old-m_new} +
+// sum e^{x-m_new}, O rescaled alike; kept unnormalised here); Tree Attention
+// article (m.srwj168.com.cn), "The energy view of attention" (max and
+// logsumexp are associative, so partial results combine in any tree).
+//
+// Work split (one launch): the (sequence, KV head) units are laid end to end as
+// a line of NT tiles of TILE tokens; CTA i takes tiles [i*NT/P, (i+1)*NT/P).  A
+// CTA that crosses a unit boundary emits one partial per unit it touched.  CTA i
+// writes unit u's partial to slot i + u: along the line both i and u only grow,
+// so i + u is unique, and unit u's partials sit in consecutive slots.
+#pragma once
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace ta {
+
+constexpr int kMaxSeqPerLaunch = 128;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLn2 = 0.693147180559945309f;
+// Lazy rescaling: a new score replaces the running max only when it exceeds it
+// by more than this (log2 units), so p = 2^(x - m) <= 2^8; the final division
+// by l cancels whichever reference max was used.
+constexpr float kRescaleThreshold = 8.0f;
+
+// Error codes recorded in the workspace error word.
+constexpr int kErrConsumerWait = 1;
+constexpr int kErrProducerWait = 2;
+constexpr int kErrDrainWait = 3;
+
+struct SplitParams {
+  const void* q;   // [B][Hq][D], this launch's first sequence
+  const void* k;   // cache base; kv_off[b] is relative to it
+  const void* v;
+  float* out;      // [B][Hq][D]
+  float* lse;      // [B][Hq]
+  int* tickets;    // [B * Hkv], zero between calls
+  float* part;     // partial slots, G * (D + 2) floats each: m[G], l[G], o[G][D]
+  int* err;        // workspace error word
+  int64_t n_tiles_total;  // NT
+  int64_t wait_limit_ns;
+  int32_t grid;           // P
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t n_q_heads;
+  float scale_log2;       // scale * log2(e): scores come out in base-2 units
+  int32_t debug_skip_tile;
+  int64_t kv_off[kMaxSeqPerLaunch];
+  int64_t seq_len[kMaxSeqPerLaunch];
+  int64_t tile_off[kMaxSeqPerLaunch + 1];  // first tile of sequence b on the line
+  int32_t n_tiles[kMaxSeqPerLaunch];       // tiles per (sequence, KV head), >= 1
+};
+
+template <typename T, int D_, int G_>
+struct SplitCfg {
+  static constexpr int D = D_;
+  static constexpr int G = G_;
+  static constexpr int ELEM = sizeof(T);
+  static constexpr int E = (G >= 8) ? 8 : 16;  // elements of a row held by one lane
+  static constexpr int LPT = D / E;            // lanes per token
+  static constexpr int TPW = 32 / LPT;         // tokens per warp step
+  static constexpr int ROW = D * ELEM;         // bytes per token row
+  static constexpr int TILE = 16384 / ROW;     // tokens per tile (16 KB of K, 16 KB of V)
+  static constexpr int NCW = 8;                // consumer warps
+  static constexpr int STEPS = TILE / (NCW * TPW);
+  static constexpr int EPC = 16 / ELEM;        // elements per 16-byte chunk
+  static constexpr int NCH = E / EPC;          // chunks per lane per row
+  static constexpr int TILE_BYTES = TILE * ROW;
+  static constexpr int NSTAGE = 4;
+  static constexpr int NCT = NCW * 32;         // consumer threads
+  static constexpr int THREADS = NCT + 32;     // + one producer warp
+  static constexpr int MERGE_BATCH = 256;      // partials whose weights are staged at once
+  static constexpr int SLOT = G * (D + 2);     // floats per partial slot
+  static constexpr int NCOL = (G * D + NCT - 1) / NCT;
+  static_assert(STEPS >= 1 && STEPS * NCW * TPW == TILE, "tile must split evenly over warps");
+  static_assert(G <= LPT, "each lane must end with one head's score");
+  static_assert(NCH >= 1 && NCH <= 4, "chunk rotation covers 1, 2 or 4 chunks");
+};
+
+template <class C>
+struct SplitSmem {
+  alignas(128) uint8_t k[C::NSTAGE][C::TILE_BYTES];
+  alignas(128) uint8_t v[C::NSTAGE][C::TILE_BYTES];
+  float wo[C::NCW][C::G][C::D];  // per-warp statistics of the current unit
+  float wm[C::NCW][C::G];
+  float wl[C::NCW][C::G];
+  float mw[C::MERGE_BATCH][C::G];  // merge weights 2^(m_c - M)
+  float mM[C::G];
+  float mL[C::G];
+  uint64_t full[C::NSTAGE];
+  uint64_t empty[C::NSTAGE];
+  int is_last;
+  int abort;
+};
+
+// ---------------------------------------------------------------------------------------------
+// Small helpers
+// ---------------------------------------------------------------------------------------------
+
+// Bounded wait on an mbarrier phase.  Gives up after limit_ns or when *abort is set.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int64_t limit_ns,
+                                           const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) return false;
+  }
+}
+
+// Head held by lane `li` of a token group after reduce_scores (see there).
+template <int G, int LPT>
+__device__ __forceinline__ int head_of_lane(int li) {
+  int h = 0;
+#pragma unroll
+  for (int half = G >> 1, off = LPT >> 1; half >= 1; half >>= 1, off >>= 1)
+    if (li & off) h += half;
+  return h;
+}
+
+template <int G, int LPT>
+__device__ __forceinline__ int lane_of_head(int g) {
+  int li = 0;
+#pragma unroll
+  for (int half = G >> 1, off = LPT >> 1; half >= 1; half >>= 1, off >>= 1)
+    if (g & half) li += off;
+  return li;
+}
+
+// Sum G per-lane partial dot products over the LPT lanes of a token group.  While
+// more than one head is left, each exchange halves the heads a lane carries (the
+// lane keeps the half selected by its lane bit and receives its partner's share of
+// it); the remaining exchanges are plain butterflies.  Afterwards the lane holds
+// the full score of head head_of_lane(li); lanes holding the same head agree bit
+// for bit (a + b == b + a).
+template <int G, int LPT>
+__device__ __forceinline__ float reduce_scores(float (&v)[G], int li) {
+  int n = G;
+#pragma unroll
+  for (int off = LPT >> 1; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const bool upper = (li & off) != 0;
+#pragma unroll
+      for (int j = 0; j < G / 2; ++j) {
+        if (j < n / 2) {
+          const float send = upper ? v[j] : v[j + n / 2];
+          const float keep = upper ? v[j + n / 2] : v[j];
+          v[j] = keep + __shfl_xor_sync(kFull, send, off);
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] += __shfl_xor_sync(kFull, v[0], off);
+    }
+  }
+  return v[0];
+}
+
+template <typename T>
+struct RowLoader;
+
+// bf16: 8 values per 16-byte chunk, widened exactly to float (bf16 is the top half of a float).
+template <>
+struct RowLoader<__nv_bfloat16> {
+  template <int NCH>
+  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float* f) {
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int c = li * NCH + ((k + rot) & (NCH - 1));
+      const uint4 w = *reinterpret_cast<const uint4*>(row + c * 16);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[k * 8 + 2 * j] = __uint_as_float(ws[j] << 16);
+        f[k * 8 + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+      }
+    }
+  }
+  __device__ __forceinline__ static float scalar(const void* base, int64_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  }
+};
+
+template <>
+struct RowLoader<float> {
+  template <int NCH>
+  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float* f) {
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int c = li * NCH + ((k + rot) & (NCH - 1));
+      const float4 w = *reinterpret_cast<const float4*>(row + c * 16);
+      f[k * 4 + 0] = w.x;
+      f[k * 4 + 1] = w.y;
+      f[k * 4 + 2] = w.z;
+      f[k * 4 + 3] = w.w;
+    }
+  }
+  __device__ __forceinline__ static float scalar(const void* base, int64_t i) {
+    return reinterpret_cast<const float*>(base)[i];
+  }
+};
+
+// Walks the tile line: unit (b, h), tile j of that unit.
+struct TileWalk {
+  int b, h;
+  int64_t j;
+  __device__ __forceinline__ void init(const SplitParams& p, int64_t t) {
+    int lo = 0, hi = p.batch - 1;  // last b with tile_off[b] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.tile_off[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    const int64_t r = t - p.tile_off[b];
+    h = static_cast<int>(r / p.n_tiles[b]);
+    j = r % p.n_tiles[b];
+  }
+  __device__ __forceinline__ void next(const SplitParams& p) {
+    if (++j == p.n_tiles[b]) {
+      j = 0;
+      if (++h == p.n_kv_heads) {
+        h = 0;
+        ++b;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ int cta_of_tile(int64_t t, int64_t NT, int P) {
+  return static_cast<int>(((t + 1) * P - 1) / NT);
+}
+
+// Sum of leaves in a fixed pairwise tree: leaf n is combined with the pending
+// subtrees as a binary counter carries, so the shape depends only on the leaf count.
+struct PairwiseSum {
+  float s[24];
+  int n = 0;
+  int top = 0;
+  __device__ __forceinline__ void push(float x) {
+    for (int c = n; c & 1; c >>= 1) x = s[--top] + x;
+    s[top++] = x;
+    ++n;
+  }
+  __device__ __forceinline__ float result() const {
+    if (top == 0) return 0.f;
+    float r = s[top - 1];
+    for (int j = top - 2; j >= 0; --j) r = s[j] + r;
+    return r;
+  }
+};
+
+__device__ __forceinline__ float tree8(const float (&a)[8]) {
+  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+}
+
+// out = O / L, lse = ln(2) (M + log2 L); an empty unit gives 0 and -inf; a unit
+// whose inputs may be incomplete (error word set) gives NaN.
+__device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq, int d, int D, float M, float L,
+                                            float O, bool write_lse) {
+  float ov, lv;
+  if (L > 0.f) {
+    ov = O / L;
+    lv = (M + log2f(L)) * kLn2;
+  } else {
+    ov = 0.f;
+    lv = -INFINITY;
+  }
+  if (*reinterpret_cast<volatile int*>(p.err) != 0) {
+    ov = __int_as_float(0x7fc00000);
+    lv = ov;
+  }
+  const int64_t row = static_cast<int64_t>(b) * p.n_q_heads + hq;
+  p.out[row * D + d] = ov;
+  if (write_lse) p.lse[row] = lv;
+}
+
+// ---------------------------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------------------------
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
+    split_kv_decode_kernel(const __grid_constant__ SplitParams p) {
+  using C = SplitCfg<T, D, G>;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SplitSmem<C>& sm = *reinterpret_cast<SplitSmem<C>*>(smem_raw);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int cta = blockIdx.x;
+  const int64_t NT = p.n_tiles_total;
+  const int64_t t_lo = static_cast<int64_t>(cta) * NT / p.grid;
+  const int64_t t_hi = static_cast<int64_t>(cta + 1) * NT / p.grid;
+  const int n_my = static_cast<int>(t_hi - t_lo);
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], C::NCW);
+    }
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &sm.abort;
+
+  if (warp == C::NCW) {
+    // ------------------------------- producer -------------------------------
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      TileWalk w;
+      w.init(p, t_lo);
+      int fills[C::NSTAGE];
+#pragma unroll
+      for (int s = 0; s < C::NSTAGE; ++s) fills[s] = 0;
+      for (int i = 0; i < n_my; ++i) {
+        const int s = i % C::NSTAGE;
+        if (i >= C::NSTAGE) {
+          if (!wait_phase(&sm.empty[s], ((i / C::NSTAGE) - 1) & 1, p.wait_limit_ns, abort_flag)) {
+            if (!*abort_flag) atomicCAS(p.err, 0, kErrProducerWait);
+            *abort_flag = 1;
+          }
+        }
+        if (*abort_flag) break;
+        const int64_t len = p.seq_len[w.b];
+        const int64_t t0 = w.j * C::TILE;
+        const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - t0));
+        if (!(cta == 0 && i == p.debug_skip_tile)) {
+          const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
+          mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+          if (bytes != 0) {
+            const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
+            bulk_load(sm.k[s], reinterpret_cast<const T*>(p.k) + off, bytes, &sm.full[s], pol);
+            bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, &sm.full[s], pol);
+          }
+          ++fills[s];
+        }
+        w.next(p);
+      }
+      // No copy may still be landing in shared memory when the CTA exits.
+#pragma unroll
+      for (int s = 0; s < C::NSTAGE; ++s) {
+        if (fills[s] > 0 && !wait_phase(&sm.full[s], (fills[s] - 1) & 1, p.wait_limit_ns, nullptr))
+          atomicCAS(p.err, 0, kErrDrainWait);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------- consumers ------------------------------
+    const int li = lane % C::LPT;
+    const int gi = lane / C::LPT;
+    const int rot = (lane / (8 / C::NCH)) % C::NCH;
+    int src_lane[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) src_lane[g] = gi * C::LPT + lane_of_head<G, C::LPT>(g);
+    auto dcol = [&](int e) {
+      const int c = li * C::NCH + (((e / C::EPC) + rot) & (C::NCH - 1));
+      return c * C::EPC + e % C::EPC;
+    };
+
+    float q[G][C::E];
+    float o[G][C::E];
+    float m = -INFINITY, l = 0.f;
+
+    auto load_q = [&](int b, int h) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const int64_t base = (static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * D;
+#pragma unroll
+        for (int e = 0; e < C::E; ++e) q[g][e] = RowLoader<T>::scalar(p.q, base + dcol(e)) * p.scale_log2;
+      }
+    };
+    auto reset = [&]() {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < C::E; ++e) o[g][e] = 0.f;
+      m = -INFINITY;
+      l = 0.f;
+    };
+
+    // Combine the statistics of every consumer lane for unit (b, h) and emit them.
+    auto finalize = [&](int b, int h) {
+      // 1) merge the TPW token groups of this warp (butterflies across groups)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mg = __shfl_sync(kFull, m, src_lane[g]);
+        const float lg = __shfl_sync(kFull, l, src_lane[g]);
+        float Mx = mg;
+#pragma unroll
+        for (int off = C::LPT; off < 32; off <<= 1) Mx = fmaxf(Mx, __shfl_xor_sync(kFull, Mx, off));
+        const float a = (mg == -INFINITY) ? 0.f : ex2(mg - Mx);
+        float ls = lg * a;
+#pragma unroll
+        for (int e = 0; e < C::E; ++e) o[g][e] *= a;
+#pragma unroll
+        for (int off = C::LPT; off < 32; off <<= 1) {
+          ls += __shfl_xor_sync(kFull, ls, off);
+#pragma unroll
+          for (int e = 0; e < C::E; ++e) o[g][e] += __shfl_xor_sync(kFull, o[g][e], off);
+        }
+        if (lane == 0) {
+          sm.wm[warp][g] = Mx;
+          sm.wl[warp][g] = ls;
+        }
+        if (gi == 0) {
+#pragma unroll
+          for (int e = 0; e < C::E; ++e) sm.wo[warp][g][dcol(e)] = o[g][e];
+        }
+      }
+      named_barrier(1, C::NCT);
+
+      // 2) merge the warps; write the final result or this CTA's partial
+      const int unit = b * p.n_kv_heads + h;
+      const int64_t U0 = p.tile_off[b] + static_cast<int64_t>(h) * p.n_tiles[b];
+      const int i_first = cta_of_tile(U0, NT, p.grid);
+      const int i_last = cta_of_tile(U0 + p.n_tiles[b] - 1, NT, p.grid);
+      const int n_parts = i_last - i_first + 1;
+      float* slot = p.part + static_cast<int64_t>(cta + unit) * C::SLOT;
+#pragma unroll
+      for (int k = 0; k < C::NCOL; ++k) {
+        const int col = tid + k * C::NCT;
+        if (col < G * D) {
+          const int g = col / D, d = col % D;
+          float Mx = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < C::NCW; ++w) Mx = fmaxf(Mx, sm.wm[w][g]);
+          float ao[8], al[8];
+#pragma unroll
+          for (int w = 0; w < C::NCW; ++w) {
+            const float mw = sm.wm[w][g];
+            const float a = (mw == -INFINITY) ? 0.f : ex2(mw - Mx);
+            ao[w] = a * sm.wo[w][g][d];
+            al[w] = a * sm.wl[w][g];
+          }
+          const float O = tree8(ao), L = tree8(al);
+          if (n_parts == 1) {
+            write_final(p, b, h * G + g, d, D, Mx, L, O, d == 0);
+          } else {
+            slot[2 * G + g * D + d] = O;
+            if (d == 0) {
+              slot[g] = Mx;
+              slot[G + g] = L;
+            }
+          }
+        }
+      }
+      if (n_parts > 1) {
+        __threadfence();
+        named_barrier(1, C::NCT);
+        if (tid == 0) sm.is_last = (atomicAdd(&p.tickets[unit], 1) == n_parts - 1);
+        named_barrier(1, C::NCT);
+        if (sm.is_last) {
+          // 3) last CTA of the unit: fixed pairwise tree over the unit's partials
+          __threadfence();
+          const float* base = p.part + static_cast<int64_t>(i_first + unit) * C::SLOT;
+          const int n = n_parts;
+          if (warp < G) {
+            float Mx = -INFINITY;
+            for (int c = lane; c < n; c += 32) Mx = fmaxf(Mx, ld_cg(base + static_cast<int64_t>(c) * C::SLOT + warp));
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) Mx = fmaxf(Mx, __shfl_xor_sync(kFull, Mx, off));
+            if (lane == 0) sm.mM[warp] = Mx;
+          }
+          named_barrier(1, C::NCT);
+          PairwiseSum acc[C::NCOL], accl[C::NCOL];
+          for (int c0 = 0; c0 < n; c0 += C::MERGE_BATCH) {
+            const int nb = min(C::MERGE_BATCH, n - c0);
+            for (int idx = tid; idx < nb * G; idx += C::NCT) {
+              const int c = idx / G, g = idx % G;
+              const float mv = ld_cg(base + static_cast<int64_t>(c0 + c) * C::SLOT + g);
+              sm.mw[c][g] = (mv == -INFINITY) ? 0.f : ex2(mv - sm.mM[g]);
+            }
+            named_barrier(1, C::NCT);
+#pragma unroll
+            for (int k = 0; k < C::NCOL; ++k) {
+              const int col = tid + k * C::NCT;
+              if (col < G * D) {
+                const int g = col / D, d = col % D;
+                for (int c = 0; c < nb; ++c) {
+                  const float* sp = base + static_cast<int64_t>(c0 + c) * C::SLOT;
+                  acc[k].push(sm.mw[c][g] * ld_cg(sp + 2 * G + g * D + d));
+                  if (d == 0) accl[k].push(sm.mw[c][g] * ld_cg(sp + G + g));
+                }
+              }
+            }
+            named_barrier(1, C::NCT);
+          }
+#pragma unroll
+          for (int k = 0; k < C::NCOL; ++k) {
+            const int col = tid + k * C::NCT;
+            if (col < G * D && col % D == 0) sm.mL[col / D] = accl[k].result();
+          }
+          named_barrier(1, C::NCT);
+#pragma unroll
+          for (int k = 0; k < C::NCOL; ++k) {
+            const int col = tid + k * C::NCT;
+            if (col < G * D) {
+              const int g = col / D, d = col % D;
+              write_final(p, b, h * G + g, d, D, sm.mM[g], sm.mL[g], acc[k].result(), d == 0);
+            }
+          }
+          if (tid == 0) p.tickets[unit] = 0;
+        }
+      }
+      named_barrier(1, C::NCT);
+    };
+
+    TileWalk w;
+    w.init(p, t_lo);
+    int cur_b = w.b, cur_h = w.h;
+    load_q(cur_b, cur_h);
+    reset();
+
+    for (int i = 0; i < n_my; ++i) {
+      if (w.b != cur_b || w.h != cur_h) {
+        finalize(cur_b, cur_h);
+        cur_b = w.b;
+        cur_h = w.h;
+        load_q(cur_b, cur_h);
+        reset();
+      }
+      const int s = i % C::NSTAGE;
+      bool ok = (*abort_flag == 0);
+      if (ok) ok = wait_phase(&sm.full[s], (i / C::NSTAGE) & 1, p.wait_limit_ns, abort_flag);
+      ok = __all_sync(kFull, ok);
+      if (!ok && lane == 0) {
+        if (!*abort_flag) atomicCAS(p.err, 0, kErrConsumerWait);
+        *abort_flag = 1;
+      }
+      if (ok) {
+        const int64_t len = p.seq_len[w.b];
+        const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - w.j * C::TILE));
+        const uint8_t* kt = sm.k[s];
+        const uint8_t* vt = sm.v[s];
+#pragma unroll
+        for (int st = 0; st < C::STEPS; ++st) {
+          const int tok = (warp * C::STEPS + st) * C::TPW + gi;
+          const bool valid = tok < nv;
+          float kf[C::E];
+          RowLoader<T>::template load<C::NCH>(kt + tok * C::ROW, li, rot, kf);
+          float sc[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < C::E; ++e) acc = fmaf(q[g][e], kf[e], acc);
+            sc[g] = acc;
+          }
+          float x = reduce_scores<G, C::LPT>(sc, li);
+          if (!valid) x = -INFINITY;
+          const bool need = x > m + kRescaleThreshold;
+          if (__any_sync(kFull, need)) {
+            const float mn = need ? x : m;
+            const float a = need ? ex2(m - mn) : 1.f;
+            l *= a;
+            m = mn;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              const float ag = __shfl_sync(kFull, a, src_lane[g]);
+#pragma unroll
+              for (int e = 0; e < C::E; ++e) o[g][e] *= ag;
+            }
+          }
+          const float pe = (x == -INFINITY) ? 0.f : ex2(x - m);
+          l += pe;
+          float pg[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) pg[g] = __shfl_sync(kFull, pe, src_lane[g]);
+          if (valid) {
+            float vf[C::E];
+            RowLoader<T>::template load<C::NCH>(vt + tok * C::ROW, li, rot, vf);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+              for (int e = 0; e < C::E; ++e) o[g][e] = fmaf(pg[g], vf[e], o[g][e]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      w.next(p);
+    }
+    if (n_my > 0) finalize(cur_b, cur_h);
+  }
+  __syncthreads();
+}
+
+}  // namespace ta

@@ -1,0 +1,569 @@
+// C ABI of the split decode-attention library (declared in include/tree_attn.h):
+// argument checks, the work plan, workspace layout and kernel launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tree_attn.h"
+#include "split_kv.cuh"
+
+namespace ta {
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+constexpr size_t kAlign = 256;
+constexpr size_t kHeaderBytes = 256;  // error word and spare
+constexpr int64_t kDefaultWaitUs = 2000000;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+ta_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int32_t>(e);
+  return TA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------
+// Kernel instances
+// ------------------------------------------------------------------------------------------
+
+struct KernelInfo {
+  void (*fn)(SplitParams);
+  size_t smem;
+  int tile;
+  int threads;
+};
+
+template <typename T, int D, int G>
+KernelInfo make_info() {
+  using C = SplitCfg<T, D, G>;
+  return KernelInfo{&split_kv_decode_kernel<T, D, G>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
+}
+
+template <typename T, int D>
+bool pick_g(int G, KernelInfo* ki) {
+  switch (G) {
+    case 1: *ki = make_info<T, D, 1>(); return true;
+    case 2: *ki = make_info<T, D, 2>(); return true;
+    case 4: *ki = make_info<T, D, 4>(); return true;
+    case 8: *ki = make_info<T, D, 8>(); return true;
+    default: return false;
+  }
+}
+
+bool pick_kernel(ta_dtype dt, int D, int G, KernelInfo* ki) {
+  if (dt == TA_BF16) {
+    if (D == 64) return pick_g<__nv_bfloat16, 64>(G, ki);
+    if (D == 128) return pick_g<__nv_bfloat16, 128>(G, ki);
+  } else if (dt == TA_F32) {
+    if (D == 64) return pick_g<float, 64>(G, ki);
+    if (D == 128) return pick_g<float, 128>(G, ki);
+  }
+  return false;
+}
+
+// Resident CTAs of an instance on the current device (sets the shared-memory opt-in once).
+ta_status resident_ctas(const KernelInfo& ki, int* device_out, int* slots_out) {
+  static std::mutex mu;
+  struct Entry {
+    int device;
+    void (*fn)(SplitParams);
+    int slots;
+  };
+  static std::vector<Entry> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lk(mu);
+  for (const Entry& c : cache)
+    if (c.device == dev && c.fn == ki.fn) {
+      *device_out = dev;
+      *slots_out = c.slots;
+      return TA_OK;
+    }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaFuncSetAttribute(reinterpret_cast<const void*>(ki.fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(ki.smem));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reinterpret_cast<const void*>(ki.fn), ki.threads,
+                                                    ki.smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (per_sm < 1) return cuda_fail(cudaErrorInvalidConfiguration);
+  cache.push_back(Entry{dev, ki.fn, sms * per_sm});
+  *device_out = dev;
+  *slots_out = sms * per_sm;
+  return TA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Work plan
+// ------------------------------------------------------------------------------------------
+
+struct Group {
+  int b0 = 0, nb = 0;
+  int P = 0;
+  int64_t NT = 0;
+  size_t tickets_off = 0, part_off = 0;  // byte offsets inside the workspace body
+  int64_t kv_off[kMaxSeqPerLaunch];
+  int64_t len[kMaxSeqPerLaunch];
+  int64_t tile_off[kMaxSeqPerLaunch + 1];
+  int32_t n_tiles[kMaxSeqPerLaunch];
+};
+
+struct Plan {
+  std::vector<Group> groups;
+  size_t body_bytes = 0;
+};
+
+// kv_offsets == nullptr: sequences packed back to back ([Hkv][S_b][D] blocks).
+// Otherwise: explicit element offset of each sequence's block (blocks may alias).
+ta_status build_plan(const int64_t* seqlens, const int64_t* kv_offsets, int batch, int Hkv, int G, int D,
+                     int tile, int slots, const ta_options* opts, Plan* plan) {
+  plan->groups.clear();
+  size_t body = 0;
+  int64_t packed = 0;
+  for (int b0 = 0; b0 < batch; b0 += kMaxSeqPerLaunch) {
+    Group g;
+    g.b0 = b0;
+    g.nb = std::min(kMaxSeqPerLaunch, batch - b0);
+    int64_t NT = 0;
+    for (int i = 0; i < g.nb; ++i) {
+      const int64_t S = seqlens[b0 + i];
+      g.len[i] = S;
+      g.kv_off[i] = kv_offsets ? kv_offsets[b0 + i] : packed;
+      packed += S * Hkv * static_cast<int64_t>(D);
+      g.n_tiles[i] = static_cast<int32_t>(std::max<int64_t>(1, (S + tile - 1) / tile));
+      g.tile_off[i] = NT;
+      NT += static_cast<int64_t>(Hkv) * g.n_tiles[i];
+    }
+    g.tile_off[g.nb] = NT;
+    g.NT = NT;
+    int64_t P = (opts && opts->num_ctas > 0) ? opts->num_ctas : slots;
+    P = std::max<int64_t>(1, std::min<int64_t>(P, NT));
+    g.P = static_cast<int>(P);
+    const int64_t units = static_cast<int64_t>(g.nb) * Hkv;
+    g.tickets_off = body;
+    body = align_up(body + sizeof(int) * units, kAlign);
+    g.part_off = body;
+    body = align_up(body + sizeof(float) * static_cast<size_t>(P + units) * G * (D + 2), kAlign);
+    plan->groups.push_back(g);
+  }
+  plan->body_bytes = body;
+  return TA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Argument checks
+// ------------------------------------------------------------------------------------------
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ta_status check_opts(const ta_options* o) {
+  if (!o) return TA_OK;
+  if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1) return TA_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i)
+    if (o->reserved[i] != 0) return TA_ERR_INVALID_ARG;
+  return TA_OK;
+}
+
+ta_status check_shape(const int64_t* seqlens, int batch, int Hq, int Hkv, int D, ta_dtype dt, KernelInfo* ki) {
+  if (batch < 0 || Hq <= 0 || Hkv <= 0) return TA_ERR_INVALID_ARG;
+  if (batch > 0 && !seqlens) return TA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TA_ERR_INVALID_ARG;
+  for (int b = 0; b < batch; ++b)
+    if (seqlens[b] < 0) return TA_ERR_INVALID_ARG;
+  if (dt != TA_BF16 && dt != TA_F32) return TA_ERR_INVALID_ARG;
+  if (!pick_kernel(dt, D, Hq / Hkv, ki)) return TA_ERR_UNSUPPORTED;
+  return TA_OK;
+}
+
+ta_status check_ptrs(const void* q, const void* k, const void* v, const float* out, const float* lse) {
+  if (!q || !k || !v || !out || !lse) return TA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return TA_ERR_INVALID_ARG;
+  if (!aligned(out, 4) || !aligned(lse, 4)) return TA_ERR_INVALID_ARG;
+  return TA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Launch of a planned decode (workspace body at `body`, error word at `err`)
+// ------------------------------------------------------------------------------------------
+
+ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, const void* k, const void* v,
+                      float* out, float* lse, int Hq, int Hkv, int D, float scale, ta_dtype dt,
+                      const ta_options* opts, uint8_t* body, int* err, cudaStream_t st) {
+  const size_t qe = (dt == TA_BF16) ? 2 : 4;
+  const double s2 = static_cast<double>(scale) * 1.4426950408889634073599246810019;
+  for (const Group& g : plan.groups) {
+    SplitParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = static_cast<const uint8_t*>(q) + static_cast<size_t>(g.b0) * Hq * D * qe;
+    p.k = k;
+    p.v = v;
+    p.out = out + static_cast<size_t>(g.b0) * Hq * D;
+    p.lse = lse + static_cast<size_t>(g.b0) * Hq;
+    p.tickets = reinterpret_cast<int*>(body + g.tickets_off);
+    p.part = reinterpret_cast<float*>(body + g.part_off);
+    p.err = err;
+    p.n_tiles_total = g.NT;
+    p.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+    p.grid = g.P;
+    p.batch = g.nb;
+    p.n_kv_heads = Hkv;
+    p.n_q_heads = Hq;
+    p.scale_log2 = static_cast<float>(s2);
+    p.debug_skip_tile = opts ? opts->debug_skip_tile : -1;
+    for (int i = 0; i < g.nb; ++i) {
+      p.kv_off[i] = g.kv_off[i];
+      p.seq_len[i] = g.len[i];
+      p.tile_off[i] = g.tile_off[i];
+      p.n_tiles[i] = g.n_tiles[i];
+    }
+    p.tile_off[g.nb] = g.tile_off[g.nb];
+    ki.fn<<<g.P, ki.threads, ki.smem, st>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return TA_OK;
+}
+
+struct DecodeArgs {
+  ta_dtype dt;
+  const void *q, *k, *v;
+  const int64_t* seqlens;
+  const int64_t* kv_offsets;
+  int batch, Hq, Hkv, D;
+  float scale;
+  float *out, *lse;
+};
+
+// Checks that need no device: options, shape, scale and (when asked) pointers.
+ta_status validate(const DecodeArgs& a, const ta_options* opts, bool check_pointers, KernelInfo* ki) {
+  ta_status s = check_opts(opts);
+  if (s != TA_OK) return s;
+  s = check_shape(a.seqlens, a.batch, a.Hq, a.Hkv, a.D, a.dt, ki);
+  if (s != TA_OK) return s;
+  if (!std::isfinite(a.scale)) return TA_ERR_INVALID_ARG;
+  if (check_pointers && a.batch > 0) return check_ptrs(a.q, a.k, a.v, a.out, a.lse);
+  return TA_OK;
+}
+
+// The work plan on the current device (queries SM count and occupancy once).
+ta_status plan_for(const DecodeArgs& a, const ta_options* opts, const KernelInfo& ki, Plan* plan) {
+  int dev = 0, slots = 1;
+  if (a.batch > 0) {
+    const ta_status s = resident_ctas(ki, &dev, &slots);
+    if (s != TA_OK) return s;
+  }
+  return build_plan(a.seqlens, a.kv_offsets, a.batch, a.Hkv, a.Hq / a.Hkv, a.D, ki.tile, slots, opts, plan);
+}
+
+ta_status decode_with_workspace(const DecodeArgs& a, const ta_options* opts, void* ws, size_t ws_bytes,
+                                cudaStream_t st) {
+  KernelInfo ki;
+  Plan plan;
+  ta_status s = validate(a, opts, true, &ki);
+  if (s != TA_OK) return s;
+  if (a.batch == 0) return TA_OK;
+  if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
+  s = plan_for(a, opts, ki, &plan);
+  if (s != TA_OK) return s;
+  if (ws_bytes < kHeaderBytes + plan.body_bytes) return TA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return launch_plan(plan, ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt, opts,
+                     base + kHeaderBytes, reinterpret_cast<int*>(base), st);
+}
+
+// Allocating form: stream-ordered allocation, zero fill, run, stream-ordered free.
+ta_status with_temp_workspace(size_t bytes, cudaStream_t st, ta_status (*run)(void*, size_t, void*, cudaStream_t),
+                              void* ctx) {
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaMemsetAsync(ws, 0, bytes, st);
+  if (e != cudaSuccess) {
+    cudaFreeAsync(ws, st);
+    return cuda_fail(e);
+  }
+  const ta_status s = run(ws, bytes, ctx, st);
+  e = cudaFreeAsync(ws, st);
+  if (s != TA_OK) return s;
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Bifurcated decode: prefix pass (all samples read the one shared prefix), suffix pass,
+// then an exact merge of the two softmax statistics per (sample, query head).
+// ------------------------------------------------------------------------------------------
+
+// out = (w_a out_a + w_b out_b) / (w_a + w_b), w_x = e^(lse_x - M), lse = M + ln(w_a + w_b).
+__global__ void merge_two_kernel(const float* __restrict__ out_a, const float* __restrict__ lse_a,
+                                 const float* __restrict__ out_b, const float* __restrict__ lse_b,
+                                 float* __restrict__ out, float* __restrict__ lse, int64_t rows, int D) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * D) return;
+  const int64_t r = i / D;
+  const int d = static_cast<int>(i % D);
+  const float la = lse_a[r], lb = lse_b[r];
+  const float M = fmaxf(la, lb);
+  float o, l;
+  if (M == -INFINITY) {
+    o = 0.f;
+    l = -INFINITY;
+  } else {
+    const float wa = (la == -INFINITY) ? 0.f : expf(la - M);
+    const float wb = (lb == -INFINITY) ? 0.f : expf(lb - M);
+    const float w = wa + wb;
+    o = (wa * out_a[i] + wb * out_b[i]) / w;
+    l = M + logf(w);
+  }
+  if (std::isnan(la) || std::isnan(lb)) o = l = __int_as_float(0x7fc00000);
+  out[i] = o;
+  if (d == 0) lse[r] = l;
+}
+
+struct BifArgs {
+  const void *q, *kp, *vp, *ks, *vs;
+  int64_t P;
+  const int64_t* suffix_lens;
+  int N, Hq, Hkv, D;
+  float scale;
+  float *out, *lse;
+};
+
+struct BifPlan {
+  KernelInfo ki;
+  Plan prefix, suffix;
+  std::vector<int64_t> prefix_lens, prefix_offs;
+  size_t scratch_off = 0, body_off = 0, suffix_off = 0, total = 0;
+};
+
+ta_status bif_validate(const BifArgs& a, const ta_options* opts, bool check_pointers, KernelInfo* ki) {
+  if (a.P < 0 || a.N < 0) return TA_ERR_INVALID_ARG;
+  if (a.N > 0 && !a.suffix_lens) return TA_ERR_INVALID_ARG;
+  const int64_t one = 0;
+  DecodeArgs probe{TA_BF16, a.q, a.kp, a.vp, &one, nullptr, a.N > 0 ? 1 : 0, a.Hq, a.Hkv, a.D, a.scale,
+                   a.out, a.lse};
+  ta_status s = validate(probe, opts, check_pointers, ki);
+  if (s != TA_OK) return s;
+  for (int n = 0; n < a.N; ++n)
+    if (a.suffix_lens[n] < 0) return TA_ERR_INVALID_ARG;
+  if (check_pointers && a.N > 0 && (!a.ks || !a.vs || !aligned(a.ks, 16) || !aligned(a.vs, 16)))
+    return TA_ERR_INVALID_ARG;
+  return TA_OK;
+}
+
+ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& ki, BifPlan* bp) {
+  bp->ki = ki;
+  bp->prefix_lens.assign(a.N, a.P);
+  bp->prefix_offs.assign(a.N, 0);
+  DecodeArgs pre{TA_BF16, a.q, a.kp, a.vp, bp->prefix_lens.data(), bp->prefix_offs.data(), a.N, a.Hq, a.Hkv, a.D,
+                 a.scale, a.out, a.lse};
+  ta_status s = plan_for(pre, opts, ki, &bp->prefix);
+  if (s != TA_OK) return s;
+  DecodeArgs suf{TA_BF16, a.q, a.ks, a.vs, a.suffix_lens, nullptr, a.N, a.Hq, a.Hkv, a.D, a.scale, a.out, a.lse};
+  s = plan_for(suf, opts, ki, &bp->suffix);
+  if (s != TA_OK) return s;
+  const size_t rows = static_cast<size_t>(a.N) * a.Hq;
+  bp->scratch_off = kHeaderBytes;
+  bp->body_off = align_up(bp->scratch_off + 2 * sizeof(float) * rows * (a.D + 1), kAlign);
+  // Each pass keeps its own tickets and partials: one pass's partials must never sit
+  // where the other pass expects zeroed tickets.
+  bp->suffix_off = align_up(bp->body_off + bp->prefix.body_bytes, kAlign);
+  bp->total = bp->suffix_off + bp->suffix.body_bytes;
+  return TA_OK;
+}
+
+ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, void* ws, size_t ws_bytes,
+                  cudaStream_t st) {
+  if (a.N == 0) return TA_OK;
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < bp.total) return TA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* err = reinterpret_cast<int*>(base);
+  const size_t rows = static_cast<size_t>(a.N) * a.Hq;
+  float* out_p = reinterpret_cast<float*>(base + bp.scratch_off);
+  float* out_s = out_p + rows * a.D;
+  float* lse_p = out_s + rows * a.D;
+  float* lse_s = lse_p + rows;
+  ta_status s = launch_plan(bp.prefix, bp.ki, a.q, a.kp, a.vp, out_p, lse_p, a.Hq, a.Hkv, a.D, a.scale, TA_BF16,
+                            opts, base + bp.body_off, err, st);
+  if (s != TA_OK) return s;
+  s = launch_plan(bp.suffix, bp.ki, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
+                  base + bp.suffix_off, err, st);
+  if (s != TA_OK) return s;
+  const int64_t n = static_cast<int64_t>(rows) * a.D;
+  merge_two_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(out_p, lse_p, out_s, lse_s, a.out,
+                                                                          a.lse, static_cast<int64_t>(rows), a.D);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TA_OK;
+}
+
+}  // namespace
+}  // namespace ta
+
+using namespace ta;
+
+extern "C" {
+
+const char* tree_attn_status_string(ta_status s) {
+  switch (s) {
+    case TA_OK: return "ok";
+    case TA_ERR_INVALID_ARG: return "invalid argument";
+    case TA_ERR_UNSUPPORTED: return "unsupported shape";
+    case TA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case TA_ERR_CUDA: return "CUDA error";
+    case TA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+  }
+  return "unknown status";
+}
+
+int32_t tree_attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+ta_status tree_attn_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                   int32_t head_dim, ta_dtype dtype, const ta_options* opts, size_t* bytes) {
+  if (!bytes) return TA_ERR_INVALID_ARG;
+  DecodeArgs a{dtype, nullptr, nullptr, nullptr, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               1.0f, nullptr, nullptr};
+  KernelInfo ki;
+  Plan plan;
+  ta_status s = validate(a, opts, false, &ki);
+  if (s != TA_OK) return s;
+  s = plan_for(a, opts, ki, &plan);
+  if (s != TA_OK) return s;
+  *bytes = kHeaderBytes + plan.body_bytes;
+  return TA_OK;
+}
+
+ta_status tree_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < kHeaderBytes) return TA_ERR_WORKSPACE;
+  const cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TA_OK;
+}
+
+ta_status tree_attn_decode_ex(ta_dtype dtype, const void* q, const void* k_cache, const void* v_cache,
+                              const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                              int32_t head_dim, float scale, float* out, float* lse, const ta_options* opts,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeArgs a{dtype, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  return decode_with_workspace(a, opts, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+struct PlainCtx {
+  DecodeArgs a;
+};
+ta_status plain_run(void* ws, size_t bytes, void* ctx, cudaStream_t st) {
+  return decode_with_workspace(static_cast<PlainCtx*>(ctx)->a, nullptr, ws, bytes, st);
+}
+ta_status decode_alloc(const DecodeArgs& a, cudaStream_t st) {
+  KernelInfo ki;
+  Plan plan;
+  ta_status s = validate(a, nullptr, true, &ki);
+  if (s != TA_OK) return s;
+  if (a.batch == 0) return TA_OK;
+  s = plan_for(a, nullptr, ki, &plan);
+  if (s != TA_OK) return s;
+  PlainCtx ctx{a};
+  return with_temp_workspace(kHeaderBytes + plan.body_bytes, st, &plain_run, &ctx);
+}
+}  // namespace
+
+ta_status tree_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                           int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale,
+                           float* out, float* lse, void* stream) {
+  DecodeArgs a{TA_BF16, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  return decode_alloc(a, static_cast<cudaStream_t>(stream));
+}
+
+ta_status tree_attn_decode_f32(const float* q, const float* k_cache, const float* v_cache, const int64_t* seqlens,
+                               int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale,
+                               float* out, float* lse, void* stream) {
+  DecodeArgs a{TA_F32, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  return decode_alloc(a, static_cast<cudaStream_t>(stream));
+}
+
+ta_status tree_attn_bifurcated_workspace_size(int64_t prefix_len, const int64_t* suffix_lens, int32_t n_samples,
+                                              int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                              const ta_options* opts, size_t* bytes) {
+  if (!bytes) return TA_ERR_INVALID_ARG;
+  BifArgs a{nullptr, nullptr, nullptr, nullptr, nullptr, prefix_len, suffix_lens, n_samples, n_q_heads,
+            n_kv_heads, head_dim, 1.0f, nullptr, nullptr};
+  KernelInfo ki;
+  ta_status s = bif_validate(a, opts, false, &ki);
+  if (s != TA_OK) return s;
+  BifPlan bp;
+  s = bif_plan(a, opts, ki, &bp);
+  if (s != TA_OK) return s;
+  *bytes = bp.total;
+  return TA_OK;
+}
+
+ta_status tree_attn_decode_bifurcated_ex(const void* q, const void* k_prefix, const void* v_prefix,
+                                         int64_t prefix_len, const void* k_suffix, const void* v_suffix,
+                                         const int64_t* suffix_lens, int32_t n_samples, int32_t n_q_heads,
+                                         int32_t n_kv_heads, int32_t head_dim, float scale, float* out, float* lse,
+                                         const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  BifArgs a{q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_len, suffix_lens, n_samples, n_q_heads,
+            n_kv_heads, head_dim, scale, out, lse};
+  KernelInfo ki;
+  ta_status s = bif_validate(a, opts, true, &ki);
+  if (s != TA_OK || n_samples == 0) return s;
+  if (!workspace || !aligned(workspace, kAlign)) return TA_ERR_WORKSPACE;
+  BifPlan bp;
+  s = bif_plan(a, opts, ki, &bp);
+  if (s != TA_OK) return s;
+  return bif_run(a, opts, bp, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+struct BifCtx {
+  BifArgs a;
+  const BifPlan* bp;
+};
+ta_status bif_alloc_run(void* ws, size_t bytes, void* ctx, cudaStream_t st) {
+  BifCtx* c = static_cast<BifCtx*>(ctx);
+  return bif_run(c->a, nullptr, *c->bp, ws, bytes, st);
+}
+}  // namespace
+
+ta_status tree_attn_decode_bifurcated(const void* q, const void* k_prefix, const void* v_prefix, int64_t prefix_len,
+                                      const void* k_suffix, const void* v_suffix, const int64_t* suffix_lens,
+                                      int32_t n_samples, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                      float scale, float* out, float* lse, void* stream) {
+  BifArgs a{q, k_prefix, v_prefix, k_suffix, v_suffix, prefix_len, suffix_lens, n_samples, n_q_heads,
+            n_kv_heads, head_dim, scale, out, lse};
+  KernelInfo ki;
+  ta_status s = bif_validate(a, nullptr, true, &ki);
+  if (s != TA_OK || n_samples == 0) return s;
+  BifPlan bp;
+  s = bif_plan(a, nullptr, ki, &bp);
+  if (s != TA_OK) return s;
+  BifCtx ctx{a, &bp};
+  return with_temp_workspace(bp.total, static_cast<cudaStream_t>(stream), &bif_alloc_run, &ctx);
+}
+
+ta_status tree_attn_check(const void* ws, void* stream) {
+  if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int word = 0;
+  e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return word == 0 ? TA_OK : TA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

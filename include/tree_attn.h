@@ -1,0 +1,172 @@
+/*
+ * tree_attn.h — exact split decode attention on one B200 (sm_100a).
+ *
+ * What it computes.  For every sequence b and query head h, with KV head
+ * g = h / (Hq / Hkv) and scores x_t = scale * q[b,h,:] . K_b[g,t,:]:
+ *
+ *     out[b,h,:] = sum_t softmax(x)_t V_b[g,t,:]         (exact softmax attention)
+ *     lse[b,h]   = ln sum_t exp(x_t)                      (natural log)
+ *
+ * following the self-attention recap S = QK^T/sqrt(d_k), P = softmax(S), O = PV
+ * of the "Attention acceleration" concept page (compassingai.com, Technical
+ * principles, part 1) for one decode query per (sequence, head).
+ *
+ * How.  The KV cache is cut into contiguous chunks, one per CTA; each chunk
+ * yields the softmax statistics (m, l, o) — running max, sum of exponentials,
+ * unnormalised output — with the online-softmax update of the same page
+ * (part 2.1, "Tiling and online softmax").  Because max and logsumexp are
+ * associative (Tree Attention article, m.srwj168.com.cn, "The energy view of
+ * attention"), the chunks' statistics are merged in a fixed log-depth pairwise
+ * tree by the last CTA to finish a (sequence, KV head); this is the on-GPU form
+ * of the query host combining softmax statistics in Star Attention's phase 2
+ * (tiaojiaomugou.com article, "Phase 2: query encoding and token generation").
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers, except `seqlens` and
+ *     `suffix_lens`, which are HOST arrays read before the call returns.
+ *   - The caller owns every buffer; the library never frees caller memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Nothing synchronises the host except
+ *     tree_attn_check().
+ *   - q, k, v pointers must be 16-byte aligned (the kernels move K/V with bulk
+ *     copies); out and lse 4-byte aligned.  Misalignment -> TA_ERR_INVALID_ARG.
+ *   - Supported shapes: head_dim in {64, 128}; G = n_q_heads / n_kv_heads in
+ *     {1, 2, 4, 8}.  Others -> TA_ERR_UNSUPPORTED.  n_q_heads % n_kv_heads != 0,
+ *     a negative length, a non-finite scale or a NULL pointer ->
+ *     TA_ERR_INVALID_ARG.  Validation errors return before anything is launched.
+ *   - A sequence of length 0 gives out = 0 and lse = -inf.
+ *   - Results are bit-identical across calls with the same shapes, lengths,
+ *     options and device (the chunking is a pure function of those; no float
+ *     atomics; fixed merge order).
+ *   - No exception crosses this interface.
+ *
+ * Layouts (row-major, no padding):
+ *   q    [B][Hq][D]       bf16 (or f32 for the _f32 entry point / TA_F32)
+ *   k, v packed per sequence: sequence b is a [Hkv][S_b][D] block; blocks are
+ *        stored back to back in batch order, so sequence b starts at element
+ *        Hkv * D * (S_0 + ... + S_{b-1}).  64-bit offsets throughout.
+ *   out  [B][Hq][D]       f32
+ *   lse  [B][Hq]          f32
+ */
+#ifndef TREE_ATTN_H
+#define TREE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TA_OK = 0,
+  TA_ERR_INVALID_ARG = 1, /* NULL / misaligned pointer, bad shape, negative length, non-finite scale */
+  TA_ERR_UNSUPPORTED = 2, /* head_dim or GQA group size without a kernel */
+  TA_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than required */
+  TA_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed; see tree_attn_last_cuda_error() */
+  TA_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out (reported by tree_attn_check) */
+} ta_status;
+
+typedef enum { TA_BF16 = 0, TA_F32 = 1 } ta_dtype;
+
+/* Optional tuning and test hooks; pass NULL for the defaults (all fields 0 / -1). */
+typedef struct {
+  int32_t num_ctas;        /* 0: one CTA per resident slot (SMs x CTAs per SM); else the split grid size */
+  int32_t wait_limit_us;   /* 0: 2,000,000 us.  Bound on every wait inside a kernel; on expiry the
+                              kernel records TA_ERR_TIMEOUT in the workspace and returns */
+  int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
+                              consumers' wait runs out (no fault: the data simply never arrives) */
+  int32_t reserved[5];     /* must be 0 */
+} ta_options;
+
+/* A short English name of a status code (static storage). */
+const char* tree_attn_status_string(ta_status status);
+
+/* The cudaError_t of the most recent TA_ERR_CUDA on this host thread (0 if none). */
+int32_t tree_attn_last_cuda_error(void);
+
+/*
+ * Workspace for tree_attn_decode_ex on the current device: a header (error word),
+ * one merge ticket per (sequence, KV head) and the chunk partials
+ * (grid + B*Hkv slots of G*(D+2) floats).  Writes the byte count to *bytes.
+ * Same argument rules as tree_attn_decode_ex.
+ */
+ta_status tree_attn_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                   int32_t head_dim, ta_dtype dtype, const ta_options* opts, size_t* bytes);
+
+/*
+ * Zero-fill a workspace on `stream`.  Required once before its first use and
+ * after any call that reported TA_ERR_TIMEOUT; every successful call leaves the
+ * tickets at zero again, so no per-call clearing is needed.
+ */
+ta_status tree_attn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Exact decode attention, bf16 q/K/V, f32 out and lse.  Allocates its workspace
+ * with cudaMallocAsync on `stream` and frees it with cudaFreeAsync, so it cannot
+ * be captured into a CUDA graph; use tree_attn_decode_ex for that.
+ * `seqlens`: host array of `batch` lengths S_b >= 0.
+ */
+ta_status tree_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                           int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale,
+                           float* out, float* lse, void* stream);
+
+/* The same for float32 q/K/V (all arithmetic is float32 on either path). */
+ta_status tree_attn_decode_f32(const float* q, const float* k_cache, const float* v_cache, const int64_t* seqlens,
+                               int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale,
+                               float* out, float* lse, void* stream);
+
+/*
+ * Decode attention with a caller-owned workspace (no allocation; one kernel
+ * launch per 128 sequences).  `workspace` must be 256-byte aligned, at least
+ * tree_attn_workspace_size() bytes, zero-filled before first use, and not used
+ * by two calls in flight at once.  `opts` may be NULL.
+ */
+ta_status tree_attn_decode_ex(ta_dtype dtype, const void* q, const void* k_cache, const void* v_cache,
+                              const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                              int32_t head_dim, float scale, float* out, float* lse, const ta_options* opts,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Bifurcated (shared-prefix) decode, after the bifurcated-attention summary
+ * (briefgpt.xyz, 2403.08845, TL;DR): sample n's query attends over the
+ * concatenation [prefix ; suffix_n] — one shared context prefilled once plus the
+ * tokens that sample decoded — computed as a prefix part and a suffix part whose
+ * softmax statistics are merged exactly.
+ *   q        [N][Hq][D] bf16
+ *   k_prefix, v_prefix  [Hkv][prefix_len][D] bf16 (one copy, shared by all samples)
+ *   k_suffix, v_suffix  packed per sample like k/v above ([Hkv][S_n][D] blocks)
+ *   suffix_lens         HOST array of N lengths >= 0
+ *   out [N][Hq][D] f32, lse [N][Hq] f32
+ * Allocates its workspace like tree_attn_decode.
+ */
+ta_status tree_attn_decode_bifurcated(const void* q, const void* k_prefix, const void* v_prefix, int64_t prefix_len,
+                                      const void* k_suffix, const void* v_suffix, const int64_t* suffix_lens,
+                                      int32_t n_samples, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                      float scale, float* out, float* lse, void* stream);
+
+/* Workspace bytes for tree_attn_decode_bifurcated_ex (same argument rules). */
+ta_status tree_attn_bifurcated_workspace_size(int64_t prefix_len, const int64_t* suffix_lens, int32_t n_samples,
+                                              int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                              const ta_options* opts, size_t* bytes);
+
+/* Bifurcated decode with a caller-owned, zero-filled workspace (rules as tree_attn_decode_ex). */
+ta_status tree_attn_decode_bifurcated_ex(const void* q, const void* k_prefix, const void* v_prefix,
+                                         int64_t prefix_len, const void* k_suffix, const void* v_suffix,
+                                         const int64_t* suffix_lens, int32_t n_samples, int32_t n_q_heads,
+                                         int32_t n_kv_heads, int32_t head_dim, float scale, float* out, float* lse,
+                                         const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
+ * Synchronise `stream` and read the workspace's error word: TA_OK, or
+ * TA_ERR_TIMEOUT if a kernel's bounded wait ran out since the workspace was
+ * last initialised (the affected outputs are NaN), or TA_ERR_CUDA.
+ */
+ta_status tree_attn_check(const void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TREE_ATTN_H */

@@ -123,6 +123,7 @@ class DecodeSpec:
     seed: int = 0
     spike_frac: float = 0.0  # fraction of keys per KV head scaled by spike_factor
     spike_factor: float = 4.0
+    scale_value: Optional[float] = None  # softmax scale; default 1/sqrt(head_dim) rounded to float32
 
     @property
     def batch(self) -> int:
@@ -130,6 +131,8 @@ class DecodeSpec:
 
     @property
     def scale(self) -> float:
+        if self.scale_value is not None:
+            return float(np.float32(self.scale_value))
         return float(np.float32(1.0 / math.sqrt(self.head_dim)))
 
     @property
