@@ -20,7 +20,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -100,53 +99,78 @@ def traffic_per_launch(spec) -> object:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """SM clock and clock-event (throttle) reasons read through NVML every 2 ms by a host
+    thread while the timed region runs (a step here lasts under a millisecond, far below
+    nvidia-smi's 200 ms sampling).  Only reads device state."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index: int):
-        self.device_index = device_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"bench_clocks_{os.getpid()}.csv")
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.idx = torch_device_index
+        self.period = period_s
+        self.samples = []
+        self.window = [None, None]
+        self.err = None
+        self._stop = False
+        self._thread = None
+
+    def _handle(self, nv):
+        import torch
+
+        try:
+            pr = torch.cuda.get_device_properties(self.idx)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _run(self):
+        import threading  # noqa: F401
+
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     int(get_reasons(h))))
+                time.sleep(self.period)
+            nv.nvmlShutdown()
+        except Exception as e:  # NVML missing or refused: report it, never fail the bench
+            self.err = f"nvml: {e}"
 
     def __enter__(self):
-        try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        import threading
+
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        time.sleep(0.05)
         return self
 
+    def start(self):
+        self.window[0] = time.perf_counter()
+
+    def stop(self):
+        self.window[1] = time.perf_counter()
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.fh.close()
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as fh:
-            for line in fh:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self.err or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+        t0, t1 = self.window
+        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1] or self.samples
+        reasons = sorted({name for _, _, r in inside for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(inside), "source": "nvml, 2 ms"}
 
 
 def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra) -> dict:
@@ -291,6 +315,7 @@ def run_gpu(args, spec) -> None:
     with ClockSampler(local_rank) as clocks:
         barrier(world)
         torch.cuda.synchronize()
+        clocks.start()
         t_begin.record(stream)
         for i in range(args.steps):
             starts[i].record(stream)
@@ -298,6 +323,7 @@ def run_gpu(args, spec) -> None:
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+        clocks.stop()
         barrier(world)
     status = ta.tree_attn_check(ws)
     if status != ta.TA_OK:
@@ -369,10 +395,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--workload", default="long_1m", choices=sorted(synth.decode_configs()))
+    workloads = {**synth.decode_configs(), **synth.capture_configs()}
+    ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
-    spec = synth.decode_configs()[args.workload]
+    spec = workloads[args.workload]
     if args.impl == "reference":
         run_reference(args, spec)
     else:

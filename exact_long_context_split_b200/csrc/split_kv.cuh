@@ -62,29 +62,61 @@ struct SplitParams {
   int32_t n_tiles[kMaxSeqPerLaunch];       // tiles per (sequence, KV head), >= 1
 };
 
-template <typename T, int D_, int G_>
+// Build-time tuning of the split kernel (defaults measured best on B200; see the design notes).
+#ifndef TA_SPLIT_WARPS
+#define TA_SPLIT_WARPS 12  // consumer warps per CTA
+#endif
+#ifndef TA_SPLIT_STAGES
+#define TA_SPLIT_STAGES 2  // depth of the shared-memory ring
+#endif
+#ifndef TA_SPLIT_ELEMS
+#define TA_SPLIT_ELEMS 8  // row elements per lane when G <= 4 (G = 8 uses half, at least one chunk)
+#endif
+#ifndef TA_SPLIT_KV_BARRIERS
+#define TA_SPLIT_KV_BARRIERS 0  // 1: separate "K landed" and "V landed" barriers per stage
+#endif
+#ifndef TA_SPLIT_TILE_BYTES
+#define TA_SPLIT_TILE_BYTES 49152  // target bytes of one K (or V) tile
+#endif
+
+constexpr int kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100 (227 KB)
+
+// G = 8 keeps 8 consumer warps: its q and o registers need more than the 128 per thread
+// that 13 resident warps leave (4 warps on one SM sub-partition).
+template <typename T, int D_, int G_, int NCW_ = (G_ >= 8 ? 8 : TA_SPLIT_WARPS), int NSTAGE_ = TA_SPLIT_STAGES>
 struct SplitCfg {
   static constexpr int D = D_;
   static constexpr int G = G_;
   static constexpr int ELEM = sizeof(T);
-  static constexpr int E = (G >= 8) ? 8 : 16;  // elements of a row held by one lane
+  static constexpr int EPC = 16 / ELEM;        // elements per 16-byte chunk
+  // Row elements held by one lane (at least one chunk; G = 8 halves it to bound registers).
+  static constexpr int E = (G >= 8) ? (TA_SPLIT_ELEMS / 2 > EPC ? TA_SPLIT_ELEMS / 2 : EPC) : TA_SPLIT_ELEMS;
+  static constexpr int E2 = E / 2;             // ... as float pairs (packed FP32 math)
   static constexpr int LPT = D / E;            // lanes per token
   static constexpr int TPW = 32 / LPT;         // tokens per warp step
   static constexpr int ROW = D * ELEM;         // bytes per token row
-  static constexpr int TILE = 16384 / ROW;     // tokens per tile (16 KB of K, 16 KB of V)
-  static constexpr int NCW = 8;                // consumer warps
-  static constexpr int STEPS = TILE / (NCW * TPW);
-  static constexpr int EPC = 16 / ELEM;        // elements per 16-byte chunk
+  static constexpr int NCW = NCW_;             // consumer warps
+  static constexpr int NSTAGE = NSTAGE_;
+  static constexpr int MERGE_BATCH = 128;      // partials whose weights are staged at once
+  // Shared memory besides the ring: per-warp statistics, merge weights, barriers and flags.
+  static constexpr int FIXED_SMEM = NCW * G * D * 4 + 2 * NCW * G * 4 + MERGE_BATCH * G * 4 + 1024;
+  static constexpr int MAX_TILE_BYTES = (kSmemLimit - FIXED_SMEM) / (2 * NSTAGE);
+  static constexpr int TILE_TARGET = TA_SPLIT_TILE_BYTES < MAX_TILE_BYTES ? TA_SPLIT_TILE_BYTES : MAX_TILE_BYTES;
+  static constexpr int STEPS_FIT = TILE_TARGET / (ROW * NCW * TPW);
+  // Tokens per warp per tile (phase length).  Longer phases give more independent work per
+  // warp but hold more registers: 8 (4 when G = 8, whose q and o take twice the registers).
+  static constexpr int MAX_STEPS = G >= 8 ? 4 : 8;
+  static constexpr int STEPS = STEPS_FIT < 1 ? 1 : (STEPS_FIT > MAX_STEPS ? MAX_STEPS : STEPS_FIT);
+  static constexpr int TILE = NCW * STEPS * TPW;  // tokens per tile (about 16 KB of K and of V)
+  static constexpr int PPC = EPC / 2;          // float pairs per chunk
   static constexpr int NCH = E / EPC;          // chunks per lane per row
   static constexpr int TILE_BYTES = TILE * ROW;
-  static constexpr int NSTAGE = 4;
   static constexpr int NCT = NCW * 32;         // consumer threads
   static constexpr int THREADS = NCT + 32;     // + one producer warp
-  static constexpr int MERGE_BATCH = 256;      // partials whose weights are staged at once
   static constexpr int SLOT = G * (D + 2);     // floats per partial slot
   static constexpr int NCOL = (G * D + NCT - 1) / NCT;
-  static_assert(STEPS >= 1 && STEPS * NCW * TPW == TILE, "tile must split evenly over warps");
   static_assert(G <= LPT, "each lane must end with one head's score");
+  static_assert(NCW >= G, "the merge uses one warp per head");
   static_assert(NCH >= 1 && NCH <= 4, "chunk rotation covers 1, 2 or 4 chunks");
 };
 
@@ -98,7 +130,8 @@ struct SplitSmem {
   float mw[C::MERGE_BATCH][C::G];  // merge weights 2^(m_c - M)
   float mM[C::G];
   float mL[C::G];
-  uint64_t full[C::NSTAGE];
+  uint64_t full[C::NSTAGE];   // K (and V, unless split) of the stage landed
+  uint64_t full_v[C::NSTAGE]; // V of the stage landed (split barriers only)
   uint64_t empty[C::NSTAGE];
   int is_last;
   int abort;
@@ -173,21 +206,19 @@ __device__ __forceinline__ float reduce_scores(float (&v)[G], int li) {
 template <typename T>
 struct RowLoader;
 
-// bf16: 8 values per 16-byte chunk, widened exactly to float (bf16 is the top half of a float).
+// bf16: 8 values per 16-byte chunk, widened exactly to float (bf16 is the top half of a
+// float), as pairs (element 2j, element 2j+1) for packed FP32 math.
 template <>
 struct RowLoader<__nv_bfloat16> {
   template <int NCH>
-  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float* f) {
+  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float2* f) {
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
       const int c = li * NCH + ((k + rot) & (NCH - 1));
       const uint4 w = *reinterpret_cast<const uint4*>(row + c * 16);
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        f[k * 8 + 2 * j] = __uint_as_float(ws[j] << 16);
-        f[k * 8 + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
-      }
+      for (int j = 0; j < 4; ++j) f[k * 4 + j] = make_float2(__uint_as_float(ws[j] << 16), __uint_as_float(ws[j] & 0xffff0000u));
     }
   }
   __device__ __forceinline__ static float scalar(const void* base, int64_t i) {
@@ -198,21 +229,42 @@ struct RowLoader<__nv_bfloat16> {
 template <>
 struct RowLoader<float> {
   template <int NCH>
-  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float* f) {
+  __device__ __forceinline__ static void load(const uint8_t* row, int li, int rot, float2* f) {
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
       const int c = li * NCH + ((k + rot) & (NCH - 1));
       const float4 w = *reinterpret_cast<const float4*>(row + c * 16);
-      f[k * 4 + 0] = w.x;
-      f[k * 4 + 1] = w.y;
-      f[k * 4 + 2] = w.z;
-      f[k * 4 + 3] = w.w;
+      f[k * 2 + 0] = make_float2(w.x, w.y);
+      f[k * 2 + 1] = make_float2(w.z, w.w);
     }
   }
   __device__ __forceinline__ static float scalar(const void* base, int64_t i) {
     return reinterpret_cast<const float*>(base)[i];
   }
 };
+
+// A lane reads its NCH chunks of a row starting at chunk `rot` (bank-conflict avoidance),
+// so register pair j holds chunk (j / PPC + rot) mod NCH of the lane's slice.  This puts
+// the pairs back in column order (pair j = columns li*E + 2j, +1) so that lanes of
+// different token groups, whose rotations differ, can be added register by register.
+template <int NCH, int PPC>
+__device__ __forceinline__ void unrotate(float2 (&a)[NCH * PPC], int rot) {
+  if constexpr (NCH > 1) {
+    float2 t[NCH * PPC];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c)
+#pragma unroll
+      for (int j = 0; j < PPC; ++j) {
+        float2 v = a[c * PPC + j];
+#pragma unroll
+        for (int r = 1; r < NCH; ++r)
+          if (rot == r) v = a[((c - r + NCH) % NCH) * PPC + j];
+        t[c * PPC + j] = v;
+      }
+#pragma unroll
+    for (int i = 0; i < NCH * PPC; ++i) a[i] = t[i];
+  }
+}
 
 // Walks the tile line: unit (b, h), tile j of that unit.
 struct TileWalk {
@@ -263,8 +315,14 @@ struct PairwiseSum {
   }
 };
 
-__device__ __forceinline__ float tree8(const float (&a)[8]) {
-  return ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+// Pairwise sum of a[OFF .. OFF+N) in a fixed balanced tree.
+template <int N, int OFF = 0, int M>
+__device__ __forceinline__ float tree_sum(const float (&a)[M]) {
+  if constexpr (N == 1) {
+    return a[OFF];
+  } else {
+    return tree_sum<N / 2, OFF>(a) + tree_sum<N - N / 2, OFF + N / 2>(a);
+  }
 }
 
 // out = O / L, lse = ln(2) (M + log2 L); an empty unit gives 0 and -inf; a unit
@@ -296,6 +354,7 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
     split_kv_decode_kernel(const __grid_constant__ SplitParams p) {
   using C = SplitCfg<T, D, G>;
+  constexpr int E2 = C::E2;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SplitSmem<C>& sm = *reinterpret_cast<SplitSmem<C>*>(smem_raw);
 
@@ -312,6 +371,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
 #pragma unroll
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.full_v[s], 1);
       mbar_init(&sm.empty[s], C::NCW);
     }
     sm.abort = 0;
@@ -343,11 +403,13 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
         const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - t0));
         if (!(cta == 0 && i == p.debug_skip_tile)) {
           const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
-          mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+          uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
+          mbar_arrive_expect_tx(&sm.full[s], TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes);
+          if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
           if (bytes != 0) {
             const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
             bulk_load(sm.k[s], reinterpret_cast<const T*>(p.k) + off, bytes, &sm.full[s], pol);
-            bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, &sm.full[s], pol);
+            bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, vbar, pol);
           }
           ++fills[s];
         }
@@ -358,39 +420,46 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
       for (int s = 0; s < C::NSTAGE; ++s) {
         if (fills[s] > 0 && !wait_phase(&sm.full[s], (fills[s] - 1) & 1, p.wait_limit_ns, nullptr))
           atomicCAS(p.err, 0, kErrDrainWait);
+        if (TA_SPLIT_KV_BARRIERS && fills[s] > 0 &&
+            !wait_phase(&sm.full_v[s], (fills[s] - 1) & 1, p.wait_limit_ns, nullptr))
+          atomicCAS(p.err, 0, kErrDrainWait);
       }
     }
     __syncwarp();
   } else {
     // ------------------------------- consumers ------------------------------
+    // Lane layout: token group gi (one token per group per step) of LPT lanes; lane li of
+    // a group holds E columns of the row (its NCH chunks, read from chunk `rot` on).
     const int li = lane % C::LPT;
     const int gi = lane / C::LPT;
     const int rot = (lane / (8 / C::NCH)) % C::NCH;
     int src_lane[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) src_lane[g] = gi * C::LPT + lane_of_head<G, C::LPT>(g);
-    auto dcol = [&](int e) {
+    auto dcol = [&](int e) {  // column of register element e (load order)
       const int c = li * C::NCH + (((e / C::EPC) + rot) & (C::NCH - 1));
       return c * C::EPC + e % C::EPC;
     };
 
-    float q[G][C::E];
-    float o[G][C::E];
-    float m = -INFINITY, l = 0.f;
+    float2 q2[G][E2];  // q * scale * log2(e), the G heads of the current KV head
+    float2 o2[G][E2];  // unnormalised output of this lane's tokens
+    float m = -INFINITY, l = 0.f;  // statistics of head head_of_lane(li) over this lane's tokens
 
     auto load_q = [&](int b, int h) {
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const int64_t base = (static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * D;
 #pragma unroll
-        for (int e = 0; e < C::E; ++e) q[g][e] = RowLoader<T>::scalar(p.q, base + dcol(e)) * p.scale_log2;
+        for (int j = 0; j < E2; ++j)
+          q2[g][j] = make_float2(RowLoader<T>::scalar(p.q, base + dcol(2 * j)) * p.scale_log2,
+                                 RowLoader<T>::scalar(p.q, base + dcol(2 * j + 1)) * p.scale_log2);
       }
     };
     auto reset = [&]() {
 #pragma unroll
       for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < C::E; ++e) o[g][e] = 0.f;
+        for (int j = 0; j < E2; ++j) o2[g][j] = make_float2(0.f, 0.f);
       m = -INFINITY;
       l = 0.f;
     };
@@ -398,6 +467,8 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
     // Combine the statistics of every consumer lane for unit (b, h) and emit them.
     auto finalize = [&](int b, int h) {
       // 1) merge the TPW token groups of this warp (butterflies across groups)
+#pragma unroll
+      for (int g = 0; g < G; ++g) unrotate<C::NCH, C::PPC>(o2[g], rot);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float mg = __shfl_sync(kFull, m, src_lane[g]);
@@ -408,12 +479,15 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
         const float a = (mg == -INFINITY) ? 0.f : ex2(mg - Mx);
         float ls = lg * a;
 #pragma unroll
-        for (int e = 0; e < C::E; ++e) o[g][e] *= a;
+        for (int j = 0; j < E2; ++j) o2[g][j] = __fmul2_rn(o2[g][j], make_float2(a, a));
 #pragma unroll
         for (int off = C::LPT; off < 32; off <<= 1) {
           ls += __shfl_xor_sync(kFull, ls, off);
 #pragma unroll
-          for (int e = 0; e < C::E; ++e) o[g][e] += __shfl_xor_sync(kFull, o[g][e], off);
+          for (int j = 0; j < E2; ++j) {
+            o2[g][j].x += __shfl_xor_sync(kFull, o2[g][j].x, off);
+            o2[g][j].y += __shfl_xor_sync(kFull, o2[g][j].y, off);
+          }
         }
         if (lane == 0) {
           sm.wm[warp][g] = Mx;
@@ -421,7 +495,10 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
         }
         if (gi == 0) {
 #pragma unroll
-          for (int e = 0; e < C::E; ++e) sm.wo[warp][g][dcol(e)] = o[g][e];
+          for (int j = 0; j < E2; ++j) {
+            sm.wo[warp][g][li * C::E + 2 * j] = o2[g][j].x;
+            sm.wo[warp][g][li * C::E + 2 * j + 1] = o2[g][j].y;
+          }
         }
       }
       named_barrier(1, C::NCT);
@@ -441,7 +518,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
           float Mx = -INFINITY;
 #pragma unroll
           for (int w = 0; w < C::NCW; ++w) Mx = fmaxf(Mx, sm.wm[w][g]);
-          float ao[8], al[8];
+          float ao[C::NCW], al[C::NCW];
 #pragma unroll
           for (int w = 0; w < C::NCW; ++w) {
             const float mw = sm.wm[w][g];
@@ -449,7 +526,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
             ao[w] = a * sm.wo[w][g][d];
             al[w] = a * sm.wl[w][g];
           }
-          const float O = tree8(ao), L = tree8(al);
+          const float O = tree_sum<C::NCW>(ao), L = tree_sum<C::NCW>(al);
           if (n_parts == 1) {
             write_final(p, b, h * G + g, d, D, Mx, L, O, d == 0);
           } else {
@@ -549,47 +626,74 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
         const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - w.j * C::TILE));
         const uint8_t* kt = sm.k[s];
         const uint8_t* vt = sm.v[s];
+        // Phase A: the scores of this warp's STEPS tokens of the tile (independent chains).
+        float x[C::STEPS];
 #pragma unroll
         for (int st = 0; st < C::STEPS; ++st) {
           const int tok = (warp * C::STEPS + st) * C::TPW + gi;
-          const bool valid = tok < nv;
-          float kf[C::E];
+          float2 kf[E2];
           RowLoader<T>::template load<C::NCH>(kt + tok * C::ROW, li, rot, kf);
           float sc[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            float acc = 0.f;
+            float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < C::E; ++e) acc = fmaf(q[g][e], kf[e], acc);
-            sc[g] = acc;
+            for (int j = 0; j < E2; ++j) acc = __ffma2_rn(q2[g][j], kf[j], acc);
+            sc[g] = acc.x + acc.y;
           }
-          float x = reduce_scores<G, C::LPT>(sc, li);
-          if (!valid) x = -INFINITY;
-          const bool need = x > m + kRescaleThreshold;
-          if (__any_sync(kFull, need)) {
-            const float mn = need ? x : m;
-            const float a = need ? ex2(m - mn) : 1.f;
-            l *= a;
-            m = mn;
+          const float xs = reduce_scores<G, C::LPT>(sc, li);
+          x[st] = (tok < nv) ? xs : -INFINITY;
+        }
+        // Phase B: one online-softmax update for the tile (lazy rescaling of m).
+        float xm = x[0];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-              const float ag = __shfl_sync(kFull, a, src_lane[g]);
+        for (int st = 1; st < C::STEPS; ++st) xm = fmaxf(xm, x[st]);
+        const bool need = xm > m + kRescaleThreshold;
+        if (__any_sync(kFull, need)) {
+          const float mn = need ? xm : m;
+          const float a = need ? ex2(m - mn) : 1.f;
+          l *= a;
+          m = mn;
 #pragma unroll
-              for (int e = 0; e < C::E; ++e) o[g][e] *= ag;
+          for (int g = 0; g < G; ++g) {
+            const float ag = __shfl_sync(kFull, a, src_lane[g]);
+#pragma unroll
+            for (int j = 0; j < E2; ++j) o2[g][j] = __fmul2_rn(o2[g][j], make_float2(ag, ag));
+          }
+        }
+        float pe[C::STEPS];
+#pragma unroll
+        for (int st = 0; st < C::STEPS; ++st) {
+          pe[st] = (x[st] == -INFINITY) ? 0.f : ex2(x[st] - m);
+          l += pe[st];
+        }
+        if (TA_SPLIT_KV_BARRIERS) {
+          bool vok = wait_phase(&sm.full_v[s], (i / C::NSTAGE) & 1, p.wait_limit_ns, abort_flag);
+          vok = __all_sync(kFull, vok);
+          if (!vok) {
+            if (lane == 0) {
+              if (!*abort_flag) atomicCAS(p.err, 0, kErrConsumerWait);
+              *abort_flag = 1;
             }
+            ok = false;
           }
-          const float pe = (x == -INFINITY) ? 0.f : ex2(x - m);
-          l += pe;
+        }
+        // Phase C: o += p v for the same tokens.
+#pragma unroll
+        for (int st = 0; st < C::STEPS; ++st) {
+          const int tok = (warp * C::STEPS + st) * C::TPW + gi;
           float pg[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) pg[g] = __shfl_sync(kFull, pe, src_lane[g]);
-          if (valid) {
-            float vf[C::E];
+          for (int g = 0; g < G; ++g) pg[g] = __shfl_sync(kFull, pe[st], src_lane[g]);
+          if (ok && tok < nv) {
+            float2 vf[E2];
             RowLoader<T>::template load<C::NCH>(vt + tok * C::ROW, li, rot, vf);
 #pragma unroll
-            for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g) {
+              const float2 pp = make_float2(pg[g], pg[g]);
 #pragma unroll
-              for (int e = 0; e < C::E; ++e) o[g][e] = fmaf(pg[g], vf[e], o[g][e]);
+              for (int j = 0; j < E2; ++j) o2[g][j] = __ffma2_rn(pp, vf[j], o2[g][j]);
+            }
           }
         }
       }

@@ -185,11 +185,20 @@ ta_status check_shape(const int64_t* seqlens, int batch, int Hq, int Hkv, int D,
   return TA_OK;
 }
 
-ta_status check_ptrs(const void* q, const void* k, const void* v, const float* out, const float* lse) {
-  if (!q || !k || !v || !out || !lse) return TA_ERR_INVALID_ARG;
+// k and v may be NULL when no token is read (every length 0); nothing dereferences them then.
+ta_status check_ptrs(const void* q, const void* k, const void* v, const float* out, const float* lse,
+                     bool kv_read) {
+  if (!q || !out || !lse) return TA_ERR_INVALID_ARG;
+  if (kv_read && (!k || !v)) return TA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16)) return TA_ERR_INVALID_ARG;
   if (!aligned(out, 4) || !aligned(lse, 4)) return TA_ERR_INVALID_ARG;
   return TA_OK;
+}
+
+bool any_tokens(const int64_t* seqlens, int batch) {
+  for (int b = 0; b < batch; ++b)
+    if (seqlens[b] > 0) return true;
+  return false;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -251,7 +260,8 @@ ta_status validate(const DecodeArgs& a, const ta_options* opts, bool check_point
   s = check_shape(a.seqlens, a.batch, a.Hq, a.Hkv, a.D, a.dt, ki);
   if (s != TA_OK) return s;
   if (!std::isfinite(a.scale)) return TA_ERR_INVALID_ARG;
-  if (check_pointers && a.batch > 0) return check_ptrs(a.q, a.k, a.v, a.out, a.lse);
+  if (check_pointers && a.batch > 0)
+    return check_ptrs(a.q, a.k, a.v, a.out, a.lse, any_tokens(a.seqlens, a.batch));
   return TA_OK;
 }
 
@@ -349,15 +359,17 @@ struct BifPlan {
 ta_status bif_validate(const BifArgs& a, const ta_options* opts, bool check_pointers, KernelInfo* ki) {
   if (a.P < 0 || a.N < 0) return TA_ERR_INVALID_ARG;
   if (a.N > 0 && !a.suffix_lens) return TA_ERR_INVALID_ARG;
-  const int64_t one = 0;
-  DecodeArgs probe{TA_BF16, a.q, a.kp, a.vp, &one, nullptr, a.N > 0 ? 1 : 0, a.Hq, a.Hkv, a.D, a.scale,
+  const int64_t plen = a.P;
+  DecodeArgs probe{TA_BF16, a.q, a.kp, a.vp, &plen, nullptr, a.N > 0 ? 1 : 0, a.Hq, a.Hkv, a.D, a.scale,
                    a.out, a.lse};
   ta_status s = validate(probe, opts, check_pointers, ki);
   if (s != TA_OK) return s;
   for (int n = 0; n < a.N; ++n)
     if (a.suffix_lens[n] < 0) return TA_ERR_INVALID_ARG;
-  if (check_pointers && a.N > 0 && (!a.ks || !a.vs || !aligned(a.ks, 16) || !aligned(a.vs, 16)))
-    return TA_ERR_INVALID_ARG;
+  if (check_pointers && a.N > 0) {
+    if (any_tokens(a.suffix_lens, a.N) && (!a.ks || !a.vs)) return TA_ERR_INVALID_ARG;
+    if (!aligned(a.ks, 16) || !aligned(a.vs, 16)) return TA_ERR_INVALID_ARG;
+  }
   return TA_OK;
 }
 

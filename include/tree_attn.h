@@ -33,7 +33,9 @@
  *   - Supported shapes: head_dim in {64, 128}; G = n_q_heads / n_kv_heads in
  *     {1, 2, 4, 8}.  Others -> TA_ERR_UNSUPPORTED.  n_q_heads % n_kv_heads != 0,
  *     a negative length, a non-finite scale or a NULL pointer ->
- *     TA_ERR_INVALID_ARG.  Validation errors return before anything is launched.
+ *     TA_ERR_INVALID_ARG (K/V pointers may be NULL only when every length they
+ *     serve is 0: nothing is read from them then).  Validation errors return
+ *     before anything is launched.
  *   - A sequence of length 0 gives out = 0 and lse = -inf.
  *   - Results are bit-identical across calls with the same shapes, lengths,
  *     options and device (the chunking is a pure function of those; no float
@@ -103,8 +105,8 @@ ta_status tree_attn_workspace_init(void* workspace, size_t workspace_bytes, void
 
 /*
  * Exact decode attention, bf16 q/K/V, f32 out and lse.  Allocates its workspace
- * with cudaMallocAsync on `stream` and frees it with cudaFreeAsync, so it cannot
- * be captured into a CUDA graph; use tree_attn_decode_ex for that.
+ * with cudaMallocAsync on `stream`, zero-fills it and frees it with cudaFreeAsync
+ * on every call; tree_attn_decode_ex takes a caller-owned workspace instead.
  * `seqlens`: host array of `batch` lengths S_b >= 0.
  */
 ta_status tree_attn_decode(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,

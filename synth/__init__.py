@@ -193,6 +193,12 @@ def decode_configs() -> Dict[str, DecodeSpec]:
     }
 
 
+def capture_configs() -> Dict[str, DecodeSpec]:
+    """Smaller versions of the long-context workload for profiler captures (same recipe,
+    1/4 of the length: 1.07 GB of K/V, still far larger than the 126 MB L2)."""
+    return {"long_256k": DecodeSpec("long_256k", [262_144], 32, 8, 128, seed=3, spike_frac=0.001)}
+
+
 def bifurcated_configs() -> Dict[str, BifurcatedSpec]:
     return {"shared_prefix": BifurcatedSpec("shared_prefix", 65_536, [256] * 64, 32, 8, 128, seed=5)}
 
