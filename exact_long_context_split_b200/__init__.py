@@ -15,6 +15,7 @@ from typing import Optional, Sequence
 from ._build import LIB, build  # noqa: F401
 
 TA_OK, TA_ERR_INVALID_ARG, TA_ERR_UNSUPPORTED, TA_ERR_WORKSPACE, TA_ERR_CUDA, TA_ERR_TIMEOUT = range(6)
+TA_ERR_SCRATCH_LIMIT = 6
 TA_BF16, TA_F32 = 0, 1
 _DTYPES = {"bf16": TA_BF16, "f32": TA_F32}
 
@@ -30,6 +31,7 @@ EXPORTED = [
     "tree_attn_bifurcated_workspace_size",
     "tree_attn_decode_bifurcated_ex",
     "tree_attn_check",
+    "tree_attn_decode_noalloc",
 ]
 
 
@@ -90,6 +92,7 @@ def lib() -> ctypes.CDLL:
                 ctypes.c_int,
             ),
             "tree_attn_check": ([vp, vp], ctypes.c_int),
+            "tree_attn_decode_noalloc": ([vp, vp, vp, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -220,3 +223,14 @@ def tree_attn_decode_bifurcated_ex(q, k_prefix, v_prefix, prefix_len, k_suffix, 
 def tree_attn_check(workspace, stream=None) -> int:
     """Synchronise the stream and return the workspace's status (TA_OK or TA_ERR_TIMEOUT); does not raise."""
     return lib().tree_attn_check(_ptr(workspace), _stream(stream, workspace))
+
+
+def tree_attn_decode_noalloc(q, k_cache, v_cache, seqlens, n_q_heads, n_kv_heads, head_dim, scale, out, lse,
+                             stream=None) -> None:
+    """tree_attn_decode without any device allocation: the library's fixed 4 MiB scratch array
+    serves as workspace (for callers that may not allocate while they run).  Calls that overlap
+    on the GPU share that array and must be serialised by the caller."""
+    arr, n = _lens(seqlens)
+    _check(lib().tree_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), arr, n, n_q_heads, n_kv_heads,
+                                          head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
+           "tree_attn_decode_noalloc")

@@ -434,6 +434,7 @@ const char* tree_attn_status_string(ta_status s) {
     case TA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case TA_ERR_CUDA: return "CUDA error";
     case TA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case TA_ERR_SCRATCH_LIMIT: return "needs more scratch than the fixed 4 MiB no-allocation buffer holds";
   }
   return "unknown status";
 }
@@ -566,6 +567,71 @@ ta_status tree_attn_decode_bifurcated(const void* q, const void* k_prefix, const
   if (s != TA_OK) return s;
   BifCtx ctx{a, &bp};
   return with_temp_workspace(bp.total, static_cast<cudaStream_t>(stream), &bif_alloc_run, &ctx);
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode without allocation: the workspace is a fixed array in the library's device memory.
+// ------------------------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr int kMaxDevices = 64;
+
+// The scratch.  In host code this name is only a stand-in for the symbol, not a device
+// address: the address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+ta_status noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return TA_OK;
+}
+
+}  // namespace
+
+ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                                   int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                   float scale, float* out, float* lse, void* stream) {
+  DecodeArgs a{TA_BF16, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  KernelInfo ki;
+  Plan plan;
+  ta_status s = validate(a, nullptr, true, &ki);
+  if (s != TA_OK) return s;
+  if (a.batch == 0) return TA_OK;
+  s = plan_for(a, nullptr, ki, &plan);
+  if (s != TA_OK) return s;
+  const size_t need = kHeaderBytes + plan.body_bytes;
+  if (need > kNoAllocScratchBytes) return TA_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  s = noalloc_scratch_address(&ws);
+  if (s != TA_OK) return s;
+  // The array keeps whatever the previous call left: clear the error word and the tickets.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  cudaError_t e = cudaMemsetAsync(base, 0, kHeaderBytes, st);
+  for (const Group& g : plan.groups) {
+    if (e != cudaSuccess) break;
+    e = cudaMemsetAsync(base + kHeaderBytes + g.tickets_off, 0, sizeof(int) * static_cast<size_t>(g.nb) * n_kv_heads,
+                        st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return launch_plan(plan, ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt, nullptr,
+                     base + kHeaderBytes, reinterpret_cast<int*>(base), st);
 }
 
 ta_status tree_attn_check(const void* ws, void* stream) {

@@ -66,7 +66,8 @@ typedef enum {
   TA_ERR_UNSUPPORTED = 2, /* head_dim or GQA group size without a kernel */
   TA_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than required */
   TA_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed; see tree_attn_last_cuda_error() */
-  TA_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out (reported by tree_attn_check) */
+  TA_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out (reported by tree_attn_check) */
+  TA_ERR_SCRATCH_LIMIT = 6 /* tree_attn_decode_noalloc: the problem needs more scratch than its fixed buffer */
 } ta_status;
 
 typedef enum { TA_BF16 = 0, TA_F32 = 1 } ta_dtype;
@@ -159,6 +160,32 @@ ta_status tree_attn_decode_bifurcated_ex(const void* q, const void* k_prefix, co
                                          int32_t n_kv_heads, int32_t head_dim, float scale, float* out, float* lse,
                                          const ta_options* opts, void* workspace, size_t workspace_bytes,
                                          void* stream);
+
+/*
+ * Decode attention that allocates nothing (no counterpart in the pages: it is a
+ * deployment variant of tree_attn_decode, same bf16 inputs, same results).
+ *
+ * For callers that cannot allocate device memory while they run: serving
+ * runtimes that carve all of HBM into their own pools at start-up and forbid
+ * other allocations, or latency-critical paths where an allocation call may
+ * block in the driver.  tree_attn_decode allocates its workspace per call and
+ * tree_attn_decode_ex needs the caller to own one; this entry point instead uses
+ * a fixed 4 MiB scratch array that the library keeps in device memory (every GPU
+ * that loads the library holds it until the process exits).
+ *
+ * The first call on each device looks up that array's device address (once per
+ * device, with the device current); make that first call before any stream
+ * capture.  Every call zero-fills the array's merge tickets and error word on
+ * `stream` before its kernel runs.  All calls share the one array, so calls that
+ * overlap on the GPU (two streams, two host threads) race and must be
+ * serialised by the caller.  A problem whose workspace would exceed 4 MiB
+ * (grid + B*Hkv partial slots of G*(D+2) floats, plus a ticket per sequence and
+ * KV head) returns TA_ERR_SCRATCH_LIMIT before anything is launched.  Other
+ * arguments and statuses as tree_attn_decode.
+ */
+ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                                   int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                   float scale, float* out, float* lse, void* stream);
 
 /*
  * Synchronise `stream` and read the workspace's error word: TA_OK, or
