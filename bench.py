@@ -86,8 +86,9 @@ def measured_peaks():
 
 
 def traffic_per_launch(spec) -> object:
-    """DRAM bytes of one launch from the committed ncu summary, scaled to this workload's KV
-    bytes; None when the kernel sources changed since the counters were taken."""
+    """DRAM bytes (read + write) of one launch from the committed ncu capture: the mean of the
+    captured launches for the captured workload, reads scaled by K/V bytes for another one.
+    None when the kernel sources changed since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as fh:
             d = json.load(fh)
@@ -95,7 +96,11 @@ def traffic_per_launch(spec) -> object:
         return None
     if d.get("kernel_hash") != kernel_hash():
         return None
-    return int(round(d["dram_bytes_per_kv_byte"] * spec.kv_bytes))
+    rd = statistics.mean(d["dram_bytes_read"])
+    wr = statistics.mean(d["dram_bytes_write"])
+    if spec.name != d["workload"]:
+        rd *= spec.kv_bytes / d["kv_bytes"]
+    return int(round(rd + wr))
 
 
 class ClockSampler:
@@ -189,8 +194,10 @@ def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra
         "data": "synthetic",
         "config": {
             "workload": spec.name,
-            "batch": spec.batch,
-            "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
+            **({"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0}
+               if isinstance(spec, synth.DecodeSpec) else
+               {"samples": spec.n_samples, "prefix_len": spec.prefix_len,
+                "suffix_len": int(max(spec.suffix_lens)) if spec.suffix_lens else 0}),
             "n_q_heads": spec.n_q_heads,
             "n_kv_heads": spec.n_kv_heads,
             "head_dim": spec.head_dim,
@@ -273,6 +280,66 @@ def run_reference(args, spec) -> None:
 # ----------------------------------------------------------------------------------------------
 
 
+class DecodeRun:
+    """Device and pinned-host buffers of one decode workload and its step (one kernel launch)."""
+
+    launches_per_step = 1
+
+    def __init__(self, spec, torch, ta):
+        self.spec, self.torch, self.ta = spec, torch, ta
+        B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+        self.seqlens = [int(s) for s in spec.seqlens]
+        inp = synth.make_decode_inputs(spec)
+        self.host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for n in ("q", "k", "v")}
+        del inp
+        self.dev = {n: t.cuda() for n, t in self.host.items()}
+        self.out = torch.empty(B, Hq, D, device="cuda")
+        self.lse = torch.empty(B, Hq, device="cuda")
+        self.ws = torch.empty(ta.tree_attn_workspace_size(self.seqlens, Hq, Hkv, D), dtype=torch.uint8, device="cuda")
+        ta.tree_attn_workspace_init(self.ws)
+        self.kv_bytes = spec.kv_bytes
+        self.tokens = spec.tokens
+        self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv}>"
+
+    def step(self, stream):
+        sp = self.spec
+        self.ta.tree_attn_decode_ex("bf16", self.dev["q"], self.dev["k"], self.dev["v"], self.seqlens, sp.n_q_heads,
+                                    sp.n_kv_heads, sp.head_dim, sp.scale, self.out, self.lse, None, self.ws,
+                                    stream=stream)
+
+
+class BifurcatedRun:
+    """Shared-prefix workload: one call = prefix pass, suffix pass and the exact merge."""
+
+    launches_per_step = 3
+
+    def __init__(self, spec, torch, ta):
+        self.spec, self.torch, self.ta = spec, torch, ta
+        N, Hq, Hkv, D = spec.n_samples, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+        self.lens = [int(s) for s in spec.suffix_lens]
+        inp = synth.make_bifurcated_inputs(spec)
+        names = ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix")
+        self.host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
+                     for n in names}
+        del inp
+        self.dev = {n: t.cuda() for n, t in self.host.items()}
+        self.out = torch.empty(N, Hq, D, device="cuda")
+        self.lse = torch.empty(N, Hq, device="cuda")
+        nbytes = ta.tree_attn_bifurcated_workspace_size(spec.prefix_len, self.lens, Hq, Hkv, D)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        ta.tree_attn_workspace_init(self.ws)
+        self.kv_bytes = spec.kv_bytes
+        self.tokens = spec.prefix_len + sum(self.lens)
+        self.kernel = "bifurcated step (prefix pass + suffix pass + merge)"
+
+    def step(self, stream):
+        sp, d = self.spec, self.dev
+        self.ta.tree_attn_decode_bifurcated_ex(d["q"], d["k_prefix"], d["v_prefix"], sp.prefix_len, d["k_suffix"],
+                                               d["v_suffix"], self.lens, sp.n_q_heads, sp.n_kv_heads, sp.head_dim,
+                                               sp.scale, self.out, self.lse, None, self.ws, stream=stream)
+
+
 def run_gpu(args, spec) -> None:
     import torch
 
@@ -287,26 +354,13 @@ def run_gpu(args, spec) -> None:
                                 device_id=torch.device("cuda", local_rank))
     import exact_long_context_split_b200 as ta
 
-    B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
-    seqlens = [int(s) for s in spec.seqlens]
-    inp = synth.make_decode_inputs(spec)
-    host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
-            for n in ("q", "k", "v")}
-    dev = {n: t.cuda() for n, t in host.items()}
-    out = torch.empty(B, Hq, D, device="cuda")
-    lse = torch.empty(B, Hq, device="cuda")
-    ws = torch.empty(ta.tree_attn_workspace_size(seqlens, Hq, Hkv, D), dtype=torch.uint8, device="cuda")
-    ta.tree_attn_workspace_init(ws)
+    run = (BifurcatedRun if isinstance(spec, synth.BifurcatedSpec) else DecodeRun)(spec, torch, ta)
     stream = torch.cuda.current_stream()
 
-    def step():
-        ta.tree_attn_decode_ex("bf16", dev["q"], dev["k"], dev["v"], seqlens, Hq, Hkv, D, spec.scale, out, lse,
-                               None, ws, stream=stream)
-
     for _ in range(args.warmup):
-        step()
+        run.step(stream)
     torch.cuda.synchronize()
-    assert ta.tree_attn_check(ws) == ta.TA_OK
+    assert ta.tree_attn_check(run.ws) == ta.TA_OK
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -319,62 +373,65 @@ def run_gpu(args, spec) -> None:
         t_begin.record(stream)
         for i in range(args.steps):
             starts[i].record(stream)
-            step()
+            run.step(stream)
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
         clocks.stop()
         barrier(world)
-    status = ta.tree_attn_check(ws)
+    status = ta.tree_attn_check(run.ws)
     if status != ta.TA_OK:
         raise RuntimeError(ta.tree_attn_status_string(status))
     elapsed_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
     kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms_per_step = elapsed_ms / args.steps
-    value = world * spec.kv_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+    value = world * run.kv_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
 
-    # End to end through the public API: pinned host -> device copies of q, K, V, the call, and
-    # the device -> host read of out and lse, every step.
+    # End to end through the public API: pinned host -> device copies of every input, the
+    # call, and the device -> host read of out and lse, every step.
     e2e_steps = max(1, min(args.steps, 5))
-    out_h = torch.empty(B, Hq, D).pin_memory()
-    lse_h = torch.empty(B, Hq).pin_memory()
+    out_h = torch.empty(run.out.shape).pin_memory()
+    lse_h = torch.empty(run.lse.shape).pin_memory()
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        for n in ("q", "k", "v"):
-            dev[n].copy_(host[n], non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        for n in run.host:
+            run.dev[n].copy_(run.host[n], non_blocking=True)
+        run.step(stream)
+        out_h.copy_(run.out, non_blocking=True)
+        lse_h.copy_(run.lse, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = sum(t.numel() * t.element_size() for t in run.host.values())
     d2h = out_h.numel() * 4 + lse_h.numel() * 4
 
     peak, peak_kind = measured_peaks()
-    achieved = spec.kv_bytes / (kernel_ms * 1e-3) / 1e9
+    achieved = run.kv_bytes / (kernel_ms * 1e-3) / 1e9
     extra = {
         "ms_per_step": ms_per_step,
         "us_per_step": ms_per_step * 1e3,
-        "kv_tokens_per_s": world * spec.tokens * args.steps / (elapsed_ms * 1e-3),
+        "kv_tokens_per_s": world * run.tokens * args.steps / (elapsed_ms * 1e-3),
         "hbm_frac_of_" + peak_kind: value / world / peak,
-        "e2e": {"value": world * spec.kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+        "e2e": {"value": world * run.kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * run.launches_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "kernel": "split_kv_decode_kernel<bf16,128,4>",
-                     "traffic": traffic_per_launch(spec)},
+                     "peak_kind": peak_kind, "kernel": run.kernel,
+                     "traffic": traffic_per_launch(spec) if isinstance(run, DecodeRun) else None},
         "clocks": clocks.summary(),
     }
-    if world == 1 and not args.no_cpu_baseline:
-        G = Hq // Hkv
+    if isinstance(run, BifurcatedRun):
+        extra["logical_kv_tokens_per_s"] = world * spec.n_samples * (spec.prefix_len + statistics.mean(run.lens)) * \
+            args.steps / (elapsed_ms * 1e-3)
+    if world == 1 and not args.no_cpu_baseline and isinstance(run, DecodeRun):
+        G = spec.n_q_heads // spec.n_kv_heads
         sec = oracle_sample_seconds(spec, 0, list(range(G)))
-        rows = B * Hq
+        rows = spec.batch * spec.n_q_heads
         cpu_val = spec.kv_bytes / (sec / G * rows) / 1e9
         extra["cpu_baseline"] = {"value": cpu_val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                  "sample": f"the {G} query heads of KV head 0 over all {spec.seqlens[0]} tokens took "
@@ -395,12 +452,14 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    workloads = {**synth.decode_configs(), **synth.capture_configs()}
+    workloads = {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs()}
     ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     spec = workloads[args.workload]
     if args.impl == "reference":
+        if isinstance(spec, synth.BifurcatedSpec):
+            raise SystemExit("the reference arm times the decode workloads")
         run_reference(args, spec)
     else:
         run_gpu(args, spec)
