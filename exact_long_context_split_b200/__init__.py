@@ -49,12 +49,17 @@ class ta_options(ctypes.Structure):
         ("num_ctas", ctypes.c_int32),
         ("wait_limit_us", ctypes.c_int32),
         ("debug_skip_tile", ctypes.c_int32),
-        ("reserved", ctypes.c_int32 * 5),
+        ("prefix_path", ctypes.c_int32),
+        ("reserved", ctypes.c_int32 * 4),
     ]
 
 
-def make_options(num_ctas: int = 0, wait_limit_us: int = 0, debug_skip_tile: int = -1) -> ta_options:
-    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, (ctypes.c_int32 * 5)())
+PREFIX_AUTO, PREFIX_TENSOR_CORE, PREFIX_SPLIT_KV = 0, 1, 2
+
+
+def make_options(num_ctas: int = 0, wait_limit_us: int = 0, debug_skip_tile: int = -1,
+                 prefix_path: int = PREFIX_AUTO) -> ta_options:
+    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, prefix_path, (ctypes.c_int32 * 4)())
 
 
 _lib = None

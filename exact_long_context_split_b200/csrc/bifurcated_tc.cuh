@@ -1,0 +1,514 @@
+// Bifurcated decode, shared-prefix part, on the 5th-generation tensor cores.
+//
+// Bifurcated attention summary (briefgpt.xyz, 2403.08845, TL;DR): when many samples
+// decode from one prefilled context, the attention over that shared context is one
+// dense product of all the samples' queries with the context keys, kept exact; the
+// samples' own decoded tokens are a second, separate product.  Per KV head h the
+// queries of every sample n and every query head g of the group form the rows
+// r = n * G + g of one matrix Q_h, so the context part is
+//     S = Q_h K_h^T,   online softmax over the context,   O = P V_h
+// ("Attention acceleration" concept page, compassingai.com, Technical principles 2.1:
+// tiles of keys, running max m and sum l, output rescaled when m grows).
+//
+// One CTA owns 128 rows (one M tile) and a contiguous chunk of 64-key tiles of the
+// context, and writes per row the statistics (m in log2 units, l, unnormalised o) of
+// its chunk; merge_prefix_suffix_kernel combines the chunks with the suffix part.
+//
+// Roles (8 warps):  warp 0 lane 0: TMA producer of K and V tiles;  warp 1: TMEM
+// allocation and lane 0 issues tcgen05.mma;  warps 2-3: convert each V tile from bf16
+// to fp16 in place (P is kept in fp16 for the P V product: bf16 P is too coarse);
+// warps 4-7: softmax, thread t owns row t = TMEM lane t.
+// TMEM columns: S buffers at 0 and 64 (fp32, 128 x 64 each), O at 128 (128 x 128).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace ta {
+
+constexpr int kBifRows = 128;       // M tile
+constexpr int kBifKeys = 64;        // keys per tile (N of S, K of P V)
+constexpr int kBifD = 128;          // head_dim
+constexpr int kBifStages = 4;       // K ring and V ring depth
+constexpr int kBifThreads = 256;
+constexpr int kBifTmemCols = 256;
+constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
+
+constexpr int kErrBifWait = 4;
+constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
+
+struct BifSmem {
+  alignas(1024) uint8_t q[2][kBifRows * 128];         // bf16 Q, two 64-column blocks, SW128 K-major
+  alignas(1024) uint8_t k[kBifStages][2][kBifKeys * 128];  // bf16 K tiles, two 64-column blocks
+  alignas(1024) uint8_t v[kBifStages][2][kBifKeys * 128];  // V tiles (bf16 -> fp16 in place), MN-major
+  alignas(1024) uint8_t p[2][kBifRows * 128];         // fp16 P, 64 keys per row, SW128 K-major
+  uint64_t k_full[kBifStages], v_full[kBifStages], v_conv[kBifStages];
+  uint64_t k_empty[kBifStages], v_empty[kBifStages];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t q_ready, mma_idle;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct BifParams {
+  const void* q;          // [N][Hq][D] bf16
+  float* part;            // [chunks][Hkv * rows_per_head][kBifPartRow]: m (log2), l, -, -, o[D]
+  int* err;
+  int n_samples;
+  int n_q_heads;
+  int n_kv_heads;
+  int rows_per_head;      // N * G
+  int n_chunks;
+  int64_t prefix_len;
+  float scale_log2;
+  int64_t wait_limit_ns;
+};
+
+// ---------------------------------------------------------------------------------------------
+// PTX wrappers (tcgen05, TMA tensor loads, proxy fences)
+// ---------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] x B[smem desc]; `accumulate` false overwrites D.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version 1.
+// lbo/sbo in bytes: for K-major operands sbo is the stride between 8-row groups (lbo unused);
+// for MN-major operands lbo is the stride between 64-element blocks of the MN dimension and
+// sbo the stride between 8-row groups of the K dimension.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3fff);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3fff) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
+  d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 with an f32 accumulator.
+// a_bf16/b_bf16: operand type (bf16 or fp16); b_mn_major: B stored MN-major.
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool a_bf16, bool b_bf16, bool b_mn_major) {
+  return (1u << 4) | ((a_bf16 ? 1u : 0u) << 7) | ((b_bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk `c` (0..7) of row `r` in a 128-byte-swizzled block of rows.
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Bounded wait shared by every role: gives up after limit_ns or once the CTA aborted.
+__device__ __forceinline__ bool bif_wait(uint64_t* bar, uint32_t parity, const BifParams& p, volatile int* abort) {
+  if (*abort) return false;
+  if (wait_phase(bar, parity, p.wait_limit_ns, abort)) return true;
+  if (!*abort) atomicCAS(p.err, 0, kErrBifWait);
+  *abort = 1;
+  return false;
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// The prefix kernel
+// ---------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kBifThreads, 1)
+    bif_prefix_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                      const __grid_constant__ BifParams p) {
+  extern __shared__ __align__(16) uint8_t bif_smem_raw[];
+  // 128-byte swizzling needs 1024-byte aligned tiles in the shared window.
+  const uint32_t raw = smem_addr(bif_smem_raw);
+  BifSmem& sm = *reinterpret_cast<BifSmem*>(bif_smem_raw + (((raw + 1023u) & ~1023u) - raw));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int mt = blockIdx.x, chunk = blockIdx.y, h = blockIdx.z;
+  const int64_t n_tiles = (p.prefix_len + kBifKeys - 1) / kBifKeys;
+  const int64_t j0 = chunk * n_tiles / p.n_chunks;
+  const int n_t = static_cast<int>((chunk + 1) * n_tiles / p.n_chunks - j0);
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kBifStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_conv[s], 64);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], 128);
+      mbar_init(&sm.p_full[b], 128);
+      mbar_init(&sm.pv_done[b], 1);
+    }
+    mbar_init(&sm.q_ready, 128);
+    mbar_init(&sm.mma_idle, 1);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sm.tmem_base)),
+                 "r"(kBifTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer -------------------------------
+    if (lane == 0) {
+      uint64_t pol;
+      asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+      int fills = 0;
+      for (int i = 0; i < n_t; ++i) {
+        const int s = i % kBifStages;
+        if (i >= kBifStages) {
+          const uint32_t par = ((i / kBifStages) - 1) & 1;
+          if (!bif_wait(&sm.k_empty[s], par, p, abort) || !bif_wait(&sm.v_empty[s], par, p, abort)) break;
+        }
+        if (*abort) break;
+        const int y = static_cast<int>(h * p.prefix_len + (j0 + i) * kBifKeys);
+        mbar_arrive_expect_tx(&sm.k_full[s], 2 * kBifKeys * 128);
+        tma_load_2d(sm.k[s][0], &kmap, 0, y, &sm.k_full[s], pol);
+        tma_load_2d(sm.k[s][1], &kmap, 64, y, &sm.k_full[s], pol);
+        mbar_arrive_expect_tx(&sm.v_full[s], 2 * kBifKeys * 128);
+        tma_load_2d(sm.v[s][0], &vmap, 0, y, &sm.v_full[s], pol);
+        tma_load_2d(sm.v[s][1], &vmap, 64, y, &sm.v_full[s], pol);
+        ++fills;
+      }
+      // Every issued copy lands before the CTA moves on (stage s was filled for tiles
+      // s, s + 4, ...; wait for the last phase of each).
+      for (int s = 0; s < kBifStages && s < fills; ++s) {
+        const int last = (fills - 1 - s) / kBifStages;  // index of the last fill of stage s
+        if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr) ||
+            !wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr))
+          atomicCAS(p.err, 0, kErrBifWait);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------- MMA issuer ---------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = f16_idesc(kBifRows, kBifKeys, true, true, false);
+      constexpr uint32_t idesc_pv = f16_idesc(kBifRows, kBifD, false, false, true);
+      const uint32_t q_base = smem_addr(sm.q);
+      const uint32_t o_tmem = tmem + 128;
+      bool ok = bif_wait(&sm.q_ready, 0, p, abort);
+      tc_fence_after();
+      for (int i = 0; ok && i <= n_t; ++i) {
+        if (i < n_t) {
+          const int s = i % kBifStages, b = i & 1;
+          ok = bif_wait(&sm.k_full[s], (i / kBifStages) & 1, p, abort);
+          if (ok && i >= 2) ok = bif_wait(&sm.s_free[b], ((i - 2) >> 1) & 1, p, abort);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_addr(sm.k[s]);
+#pragma unroll
+          for (int kk = 0; kk < kBifD / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
+            const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
+            const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
+            tc_mma_f16(tmem + b * kBifKeys, a, bd, idesc_qk, kk > 0);
+          }
+          tc_commit(&sm.k_empty[s]);
+          tc_commit(&sm.s_full[b]);
+        }
+        if (i >= 1) {
+          const int jj = i - 1, s2 = jj % kBifStages, b2 = jj & 1;
+          ok = bif_wait(&sm.p_full[b2], (jj >> 1) & 1, p, abort);
+          if (ok) ok = bif_wait(&sm.v_conv[s2], (jj / kBifStages) & 1, p, abort);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t p_base = smem_addr(sm.p[b2]);
+          const uint32_t v_base = smem_addr(sm.v[s2]);
+#pragma unroll
+          for (int kk = 0; kk < kBifKeys / 16; ++kk) {
+            const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
+            tc_mma_f16(o_tmem, a, bd, idesc_pv, jj > 0 || kk > 0);
+          }
+          tc_commit(&sm.v_empty[s2]);
+          tc_commit(&sm.pv_done[b2]);
+        }
+      }
+      // Every issued MMA completes before the tensor memory is released.
+      tc_commit(&sm.mma_idle);
+      if (!wait_phase(&sm.mma_idle, 0, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------- V converters -------------------------------
+    const int ct = tid - 64;
+    for (int i = 0; i < n_t; ++i) {
+      const int s = i % kBifStages;
+      if (!bif_wait(&sm.v_full[s], (i / kBifStages) & 1, p, abort)) break;
+      uint4* v4 = reinterpret_cast<uint4*>(sm.v[s]);
+#pragma unroll 4
+      for (int c = ct; c < 2 * kBifKeys * 128 / 16; c += 64) {
+        uint4 w = v4[c];
+        uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __half2 hv =
+              __floats2half2_rn(__uint_as_float(ws[e] << 16), __uint_as_float(ws[e] & 0xffff0000u));
+          ws[e] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        v4[c] = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.v_conv[s]);
+    }
+  } else {
+    // ------------------------------- softmax ------------------------------------
+    const int r = tid - 128;                          // row of the M tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int G = p.n_q_heads / p.n_kv_heads;
+    const int row = mt * kBifRows + r;                // row of this KV head's query matrix
+    const bool valid_row = row < p.rows_per_head;
+    {
+      const int n = row / G, g = row % G;
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.q) +
+                                                        (static_cast<int64_t>(n) * p.n_q_heads + h * G + g) * kBifD);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 w = valid_row ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm.q[c >> 3] + sw128_offset(r, c & 7)) = w;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.q_ready);
+    }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; ok && i < n_t; ++i) {
+      const int b = i & 1;
+      ok = bif_wait(&sm.s_full[b], (i >> 1) & 1, p, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      float x[kBifKeys];
+      {
+        float t[32];
+        tmem_ld32(tmem + lane_base + b * kBifKeys, t);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = t[c];
+        tmem_ld32(tmem + lane_base + b * kBifKeys + 32, t);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[32 + c] = t[c];
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[b]);
+      const int64_t nvalid = p.prefix_len - (j0 + i) * kBifKeys;
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBifKeys; ++c) {
+        x[c] = (c < nvalid) ? x[c] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, x[c]);
+      }
+      const bool need = tmax > m + kBifRescale;
+      const float mn = need ? tmax : m;
+      float rs = 0.f;
+      uint32_t ph[kBifKeys / 2];
+#pragma unroll
+      for (int c = 0; c < kBifKeys; c += 2) {
+        const float p0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn);
+        const float p1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn);
+        rs += p0 + p1;
+        const __half2 hv = __floats2half2_rn(p0, p1);
+        ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+      // P buffer b was last read by the P V product of tile i - 2.
+      if (i >= 2) ok = bif_wait(&sm.pv_done[b], ((i - 2) >> 1) & 1, p, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(sm.p[b] + sw128_offset(r, c)) =
+            make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
+      fence_proxy_async_smem();
+      const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
+      // O holds tiles 0..i-1: rescale it (after the P V product of tile i-1) when m grew.
+      if (__any_sync(0xffffffffu, need && i >= 1)) {
+        ok = bif_wait(&sm.pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, p, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int q4 = 0; q4 < kBifD / 32; ++q4) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + 128 + q4 * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] *= alpha;
+          tmem_st32(tmem + lane_base + 128 + q4 * 32, o);
+        }
+        tmem_wait_st();
+      }
+      l = l * alpha + rs;
+      m = mn;
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[b]);
+    }
+    // The chunk's statistics of this row.
+    float* dst = p.part + ((static_cast<int64_t>(chunk) * p.n_kv_heads + h) * p.rows_per_head + row) * kBifPartRow;
+    if (n_t > 0 && ok) {
+      ok = bif_wait(&sm.pv_done[(n_t - 1) & 1], ((n_t - 1) >> 1) & 1, p, abort);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (n_t > 0 && ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int q4 = 0; q4 < kBifD / 32; ++q4) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + 128 + q4 * 32, o);
+        tmem_wait_ld();
+        if (valid_row) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + 4 + q4 * 32 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        }
+      }
+      if (valid_row) {
+        dst[0] = m;
+        dst[1] = l;
+      }
+    } else if (valid_row) {
+      // Empty chunk, or an aborted one (the error word is set and the merge writes NaN).
+      dst[0] = -INFINITY;
+      dst[1] = 0.f;
+      for (int c = 0; c < kBifD; ++c) dst[4 + c] = 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kBifTmemCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Merge: the prefix chunks' statistics with the suffix result, per (sample, query head)
+// ---------------------------------------------------------------------------------------------
+
+// Suffix part given normalised (out_s, lse_s); it enters as m = lse_s log2(e), l = 1, o = out_s.
+__global__ void merge_prefix_suffix_kernel(const float* __restrict__ part, int n_chunks, int n_kv_heads,
+                                           int rows_per_head, const float* __restrict__ out_s,
+                                           const float* __restrict__ lse_s, float* __restrict__ out,
+                                           float* __restrict__ lse, int n_samples, int n_q_heads,
+                                           const int* __restrict__ err) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(n_samples) * n_q_heads * kBifD;
+  if (i >= total) return;
+  const int d = static_cast<int>(i % kBifD);
+  const int64_t rq = i / kBifD;  // n * Hq + hq
+  const int n = static_cast<int>(rq / n_q_heads), hq = static_cast<int>(rq % n_q_heads);
+  const int G = n_q_heads / n_kv_heads;
+  const int h = hq / G, g = hq % G;
+  const int64_t prow = static_cast<int64_t>(h) * rows_per_head + n * G + g;
+  const int64_t stride = static_cast<int64_t>(n_kv_heads) * rows_per_head * kBifPartRow;
+  const float ls = lse_s[rq];
+  const float ms = (ls == -INFINITY) ? -INFINITY : ls * 1.44269504088896340736f;
+  float M = ms;
+  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, part[c * stride + prow * kBifPartRow]);
+  float L = 0.f, O = 0.f;
+  if (M != -INFINITY) {
+    for (int c = 0; c < n_chunks; ++c) {
+      const float* pc = part + c * stride + prow * kBifPartRow;
+      const float w = (pc[0] == -INFINITY) ? 0.f : ex2(pc[0] - M);
+      L += w * pc[1];
+      O += w * pc[4 + d];
+    }
+    const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+    L += w;
+    O += w * out_s[rq * kBifD + d];
+  }
+  float ov = 0.f, lv = -INFINITY;
+  if (L > 0.f) {
+    ov = O / L;
+    lv = (M + log2f(L)) * 0.693147180559945309f;
+  }
+  if (*reinterpret_cast<const volatile int*>(err) != 0 || ls != ls) ov = lv = __int_as_float(0x7fc00000);
+  out[rq * kBifD + d] = ov;
+  if (d == 0) lse[rq] = lv;
+}
+
+}  // namespace ta

@@ -79,4 +79,18 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
 
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
+// Bounded wait on an mbarrier phase.  Gives up after limit_ns or when *abort is set.
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int64_t limit_ns,
+                                           const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) return false;
+  }
+}
+
 }  // namespace ta

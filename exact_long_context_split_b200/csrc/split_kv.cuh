@@ -141,20 +141,6 @@ struct SplitSmem {
 // Small helpers
 // ---------------------------------------------------------------------------------------------
 
-// Bounded wait on an mbarrier phase.  Gives up after limit_ns or when *abort is set.
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, int64_t limit_ns,
-                                           const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (static_cast<int64_t>(global_timer_ns() - t0) > limit_ns) return false;
-  }
-}
-
 // Head held by lane `li` of a token group after reduce_scores (see there).
 template <int G, int LPT>
 __device__ __forceinline__ int head_of_lane(int li) {

@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "../../include/tree_attn.h"
+#include "bifurcated_tc.cuh"
 #include "split_kv.cuh"
 
 namespace ta {
@@ -169,7 +170,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 ta_status check_opts(const ta_options* o) {
   if (!o) return TA_OK;
   if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1) return TA_ERR_INVALID_ARG;
-  for (int i = 0; i < 5; ++i)
+  if (o->prefix_path < 0 || o->prefix_path > 2) return TA_ERR_INVALID_ARG;
+  for (int i = 0; i < 4; ++i)
     if (o->reserved[i] != 0) return TA_ERR_INVALID_ARG;
   return TA_OK;
 }
@@ -354,7 +356,58 @@ struct BifPlan {
   Plan prefix, suffix;
   std::vector<int64_t> prefix_lens, prefix_offs;
   size_t scratch_off = 0, body_off = 0, suffix_off = 0, total = 0;
+  // tensor-core prefix pass
+  bool tc = false;
+  int mtiles = 0, chunks = 0, rows_per_head = 0;
+  size_t part_off = 0;
 };
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [rows][128] bf16 matrix, 64 x 64 boxes, 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* map, const void* base, int64_t rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn || rows <= 0 || rows >= (int64_t(1) << 31)) return false;  // tile rows are 32-bit coordinates
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kBifD), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kBifD) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBifKeys)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+ta_status bif_tc_setup(int* sms) {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(BifSmem) + 1024));
+  });
+  if (err != cudaSuccess) return cuda_fail(err);
+  return TA_OK;
+}
 
 ta_status bif_validate(const BifArgs& a, const ta_options* opts, bool check_pointers, KernelInfo* ki) {
   if (a.P < 0 || a.N < 0) return TA_ERR_INVALID_ARG;
@@ -391,6 +444,25 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
   // where the other pass expects zeroed tickets.
   bp->suffix_off = align_up(bp->body_off + bp->prefix.body_bytes, kAlign);
   bp->total = bp->suffix_off + bp->suffix.body_bytes;
+  // Tensor-core prefix pass: one CTA per (128-row tile, prefix chunk, KV head).
+  const int path = opts ? opts->prefix_path : 0;
+  const bool tc_shape = a.D == kBifD && a.P > 0;
+  if (path == 1 && !tc_shape) return TA_ERR_UNSUPPORTED;
+  if (path != 2 && tc_shape && a.N > 0) {
+    int sms = 0;
+    s = bif_tc_setup(&sms);
+    if (s != TA_OK) return s;
+    bp->tc = true;
+    bp->rows_per_head = a.N * (a.Hq / a.Hkv);
+    bp->mtiles = (bp->rows_per_head + kBifRows - 1) / kBifRows;
+    const int64_t tiles = (a.P + kBifKeys - 1) / kBifKeys;
+    int64_t chunks = sms / (static_cast<int64_t>(bp->mtiles) * a.Hkv);
+    chunks = std::max<int64_t>(1, std::min<int64_t>(chunks, tiles));
+    bp->chunks = static_cast<int>(chunks);
+    bp->part_off = align_up(bp->total, kAlign);
+    bp->total = bp->part_off +
+                sizeof(float) * static_cast<size_t>(chunks) * a.Hkv * bp->rows_per_head * kBifPartRow;
+  }
   return TA_OK;
 }
 
@@ -405,8 +477,42 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
   float* out_s = out_p + rows * a.D;
   float* lse_p = out_s + rows * a.D;
   float* lse_s = lse_p + rows;
-  ta_status s = launch_plan(bp.prefix, bp.ki, a.q, a.kp, a.vp, out_p, lse_p, a.Hq, a.Hkv, a.D, a.scale, TA_BF16,
-                            opts, base + bp.body_off, err, st);
+  ta_status s;
+  if (bp.tc) {
+    CUtensorMap kmap, vmap;
+    const int64_t kv_rows = static_cast<int64_t>(a.Hkv) * a.P;
+    const bool maps = encode_kv_map(&kmap, a.kp, kv_rows) && encode_kv_map(&vmap, a.vp, kv_rows);
+    if (maps) {
+      BifParams bpp;
+      bpp.q = a.q;
+      bpp.part = reinterpret_cast<float*>(base + bp.part_off);
+      bpp.err = err;
+      bpp.n_samples = a.N;
+      bpp.n_q_heads = a.Hq;
+      bpp.n_kv_heads = a.Hkv;
+      bpp.rows_per_head = bp.rows_per_head;
+      bpp.n_chunks = bp.chunks;
+      bpp.prefix_len = a.P;
+      bpp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
+      bpp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+      const dim3 grid(bp.mtiles, bp.chunks, a.Hkv);
+      bif_prefix_kernel<<<grid, kBifThreads, sizeof(BifSmem) + 1024, st>>>(kmap, vmap, bpp);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e);
+      s = launch_plan(bp.suffix, bp.ki, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
+                      base + bp.suffix_off, err, st);
+      if (s != TA_OK) return s;
+      const int64_t n = static_cast<int64_t>(rows) * a.D;
+      merge_prefix_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+          bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse, a.N, a.Hq, err);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e);
+      return TA_OK;
+    }
+    if (opts && opts->prefix_path == 1) return TA_ERR_UNSUPPORTED;
+  }
+  s = launch_plan(bp.prefix, bp.ki, a.q, a.kp, a.vp, out_p, lse_p, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
+                  base + bp.body_off, err, st);
   if (s != TA_OK) return s;
   s = launch_plan(bp.suffix, bp.ki, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                   base + bp.suffix_off, err, st);

@@ -79,7 +79,10 @@ typedef struct {
                               kernel records TA_ERR_TIMEOUT in the workspace and returns */
   int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
                               consumers' wait runs out (no fault: the data simply never arrives) */
-  int32_t reserved[5];     /* must be 0 */
+  int32_t prefix_path;     /* bifurcated calls only.  0: automatic (tensor-core prefix pass when
+                              head_dim is 128 and the prefix is not empty); 1: tensor-core pass
+                              (TA_ERR_UNSUPPORTED if not possible); 2: split-KV pass per sample */
+  int32_t reserved[4];     /* must be 0 */
 } ta_options;
 
 /* A short English name of a status code (static storage). */

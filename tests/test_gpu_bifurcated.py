@@ -9,7 +9,7 @@ from gpu_util import compare, device_tensor, empty_outputs, new_workspace
 pytestmark = pytest.mark.gpu
 
 
-def bif_gpu(inp, sp, entry="ex"):
+def bif_gpu(inp, sp, entry="ex", prefix_path=0):
     import torch
 
     import exact_long_context_split_b200 as ta
@@ -21,8 +21,9 @@ def bif_gpu(inp, sp, entry="ex"):
     out, lse = empty_outputs(N, Hq, D)
     lens = [int(s) for s in sp.suffix_lens]
     if entry == "ex":
-        ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(P, lens, Hq, Hkv, D))
-        ta.tree_attn_decode_bifurcated_ex(q, kp, vp, P, ks, vs, lens, Hq, Hkv, D, sp.scale, out, lse, None, ws)
+        opts = ta.make_options(prefix_path=prefix_path)
+        ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(P, lens, Hq, Hkv, D, opts))
+        ta.tree_attn_decode_bifurcated_ex(q, kp, vp, P, ks, vs, lens, Hq, Hkv, D, sp.scale, out, lse, opts, ws)
         assert ta.tree_attn_check(ws) == ta.TA_OK
     else:
         ta.tree_attn_decode_bifurcated(q, kp, vp, P, ks, vs, lens, Hq, Hkv, D, sp.scale, out, lse)
@@ -53,6 +54,44 @@ def test_bifurcated_small(prefix_len, suffix_lens, Hq, Hkv, D, entry):
     compare(out, lse, *oracle_bif(inp, sp))
 
 
+# Tensor-core prefix pass (prefix_path 1) and the split-KV pass per sample (2) on shapes with
+# several 128-row tiles (N * G > 128), a partial last row tile, partial 64-key tiles, one tile,
+# and more chunks than tiles.
+TC_CASES = [
+    (65, [3, 70], 8, 2, 128),          # 8 rows, 2 key tiles (one partial)
+    (1000, [5, 0, 64, 130], 32, 8, 128),
+    (4097, [1] * 40, 16, 4, 128),      # 160 rows: two row tiles, the second partial
+    (300, [9] * 64, 16, 2, 128),       # 512 rows: four row tiles
+    (64, [0, 2], 8, 8, 128),           # G = 1, exactly one key tile
+    (12345, [100] * 20, 32, 8, 128),
+]
+
+
+@pytest.mark.parametrize("prefix_path", [1, 2])
+@pytest.mark.parametrize("prefix_len,suffix_lens,Hq,Hkv,D", TC_CASES)
+def test_bifurcated_prefix_paths(prefix_len, suffix_lens, Hq, Hkv, D, prefix_path):
+    sp = synth.BifurcatedSpec("case", prefix_len, suffix_lens, Hq, Hkv, D, seed=23)
+    inp = synth.make_bifurcated_inputs(sp)
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path)
+    compare(out, lse, *oracle_bif(inp, sp))
+
+
+def test_tensor_core_prefix_is_deterministic():
+    sp = synth.BifurcatedSpec("case", 20000, [50] * 32, 32, 8, 128, seed=24)
+    inp = synth.make_bifurcated_inputs(sp)
+    a = bif_gpu(inp, sp, "ex", 1)
+    b = bif_gpu(inp, sp, "ex", 1)
+    assert np.array_equal(a[0].view(np.uint32), b[0].view(np.uint32))
+    assert np.array_equal(a[1].view(np.uint32), b[1].view(np.uint32))
+
+
+def test_tensor_core_prefix_unsupported_shape():
+    import exact_long_context_split_b200 as ta
+
+    with pytest.raises(ta.TreeAttnError):
+        ta.tree_attn_bifurcated_workspace_size(100, [1, 2], 8, 2, 64, ta.make_options(prefix_path=1))
+
+
 def test_bifurcated_equals_plain_decode_of_concatenation():
     """Exactness of the split: the GPU bifurcated result matches the GPU plain decode over
     [prefix ; suffix_n] (both checked against the oracle)."""
@@ -63,10 +102,11 @@ def test_bifurcated_equals_plain_decode_of_concatenation():
     compare(out, lse, *ref)
 
 
-def test_bifurcated_config_sampled():
+@pytest.mark.parametrize("prefix_path", [1, 2])
+def test_bifurcated_config_sampled(prefix_path):
     sp = synth.bifurcated_configs()["shared_prefix"]
     inp = synth.make_bifurcated_inputs(sp)
-    out, lse = bif_gpu(inp, sp)
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
     pairs = [(0, 0), (17, 9), (40, 22), (63, 31)]
     compare(out, lse, *oracle_bif(inp, sp, pairs=pairs), pairs=pairs)
