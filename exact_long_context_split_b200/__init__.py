@@ -50,16 +50,20 @@ class ta_options(ctypes.Structure):
         ("wait_limit_us", ctypes.c_int32),
         ("debug_skip_tile", ctypes.c_int32),
         ("prefix_path", ctypes.c_int32),
-        ("reserved", ctypes.c_int32 * 4),
+        ("split_tiles", ctypes.c_int32),
+        ("reserved", ctypes.c_int32 * 3),
     ]
 
 
 PREFIX_AUTO, PREFIX_TENSOR_CORE, PREFIX_SPLIT_KV = 0, 1, 2
 
 
+TILES_AUTO, TILES_LONG, TILES_SHORT = 0, 1, 2
+
+
 def make_options(num_ctas: int = 0, wait_limit_us: int = 0, debug_skip_tile: int = -1,
-                 prefix_path: int = PREFIX_AUTO) -> ta_options:
-    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, prefix_path, (ctypes.c_int32 * 4)())
+                 prefix_path: int = PREFIX_AUTO, split_tiles: int = TILES_AUTO) -> ta_options:
+    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, prefix_path, split_tiles, (ctypes.c_int32 * 3)())
 
 
 _lib = None

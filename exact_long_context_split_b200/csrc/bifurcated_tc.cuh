@@ -10,15 +10,17 @@
 // ("Attention acceleration" concept page, compassingai.com, Technical principles 2.1:
 // tiles of keys, running max m and sum l, output rescaled when m grows).
 //
-// One CTA owns 128 rows (one M tile) and a contiguous chunk of 64-key tiles of the
-// context, and writes per row the statistics (m in log2 units, l, unnormalised o) of
-// its chunk; merge_prefix_suffix_kernel combines the chunks with the suffix part.
+// Each CTA writes per row the statistics (m in log2 units, l, unnormalised o) of its
+// chunk; merge_prefix_suffix_kernel combines the chunks with the suffix part.
 //
-// Roles (8 warps):  warp 0 lane 0: TMA producer of K and V tiles;  warp 1: TMEM
+// One CTA owns up to 256 rows (two M tiles of 128) and a contiguous chunk of 64-key
+// tiles of the context; both M tiles consume every K/V tile it loads.
+// Roles (12 warps):  warp 0 lane 0: TMA producer of K and V tiles;  warp 1: TMEM
 // allocation and lane 0 issues tcgen05.mma;  warps 2-3: convert each V tile from bf16
 // to fp16 in place (P is kept in fp16 for the P V product: bf16 P is too coarse);
-// warps 4-7: softmax, thread t owns row t = TMEM lane t.
-// TMEM columns: S buffers at 0 and 64 (fp32, 128 x 64 each), O at 128 (128 x 128).
+// warps 4-7 and 8-11: softmax of M tile 0 and 1, thread t owns row t = TMEM lane t.
+// TMEM columns: S of tile w, buffer b at 128 w + 64 b (fp32, 128 x 64); O of tile w at
+// 256 + 128 w (128 x 128).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -30,25 +32,26 @@
 
 namespace ta {
 
-constexpr int kBifRows = 128;       // M tile
+constexpr int kBifRows = 128;       // rows of one M tile (one TMEM lane each)
+constexpr int kBifMT = 2;           // M tiles per CTA: the CTA's 256 rows share every K/V tile
 constexpr int kBifKeys = 64;        // keys per tile (N of S, K of P V)
 constexpr int kBifD = 128;          // head_dim
-constexpr int kBifStages = 4;       // K ring and V ring depth
-constexpr int kBifThreads = 256;
-constexpr int kBifTmemCols = 256;
+constexpr int kBifStages = 3;       // K ring and V ring depth
+constexpr int kBifThreads = 384;    // 12 warps
+constexpr int kBifTmemCols = 512;   // S: 2 tiles x 2 buffers x 64 columns; O: 2 tiles x 128 columns
 constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
 
 constexpr int kErrBifWait = 4;
 constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
 
 struct BifSmem {
-  alignas(1024) uint8_t q[2][kBifRows * 128];         // bf16 Q, two 64-column blocks, SW128 K-major
+  alignas(1024) uint8_t q[kBifMT][2][kBifRows * 128];      // bf16 Q tiles, two 64-column blocks each, SW128
   alignas(1024) uint8_t k[kBifStages][2][kBifKeys * 128];  // bf16 K tiles, two 64-column blocks
   alignas(1024) uint8_t v[kBifStages][2][kBifKeys * 128];  // V tiles (bf16 -> fp16 in place), MN-major
-  alignas(1024) uint8_t p[2][kBifRows * 128];         // fp16 P, 64 keys per row, SW128 K-major
+  alignas(1024) uint8_t p[kBifMT][2][kBifRows * 128];      // fp16 P per M tile, double buffered, SW128
   uint64_t k_full[kBifStages], v_full[kBifStages], v_conv[kBifStages];
   uint64_t k_empty[kBifStages], v_empty[kBifStages];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t s_full[kBifMT][2], s_free[kBifMT][2], p_full[kBifMT][2], pv_done[kBifMT][2];
   uint64_t q_ready, mma_idle;
   uint32_t tmem_base;
   int abort;
@@ -194,7 +197,9 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int mt = blockIdx.x, chunk = blockIdx.y, h = blockIdx.z;
+  const int chunk = blockIdx.y, h = blockIdx.z;
+  const int row0 = blockIdx.x * kBifMT * kBifRows;  // first row of this CTA in the head's query matrix
+  const int n_mt = min(kBifMT, (p.rows_per_head - row0 + kBifRows - 1) / kBifRows);  // active M tiles
   const int64_t n_tiles = (p.prefix_len + kBifKeys - 1) / kBifKeys;
   const int64_t j0 = chunk * n_tiles / p.n_chunks;
   const int n_t = static_cast<int>((chunk + 1) * n_tiles / p.n_chunks - j0);
@@ -209,13 +214,15 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       mbar_init(&sm.v_empty[s], 1);
     }
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], 128);
-      mbar_init(&sm.p_full[b], 128);
-      mbar_init(&sm.pv_done[b], 1);
-    }
-    mbar_init(&sm.q_ready, 128);
+    for (int w = 0; w < kBifMT; ++w)
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.s_full[w][b], 1);
+        mbar_init(&sm.s_free[w][b], kBifRows);
+        mbar_init(&sm.p_full[w][b], kBifRows);
+        mbar_init(&sm.pv_done[w][b], 1);
+      }
+    mbar_init(&sm.q_ready, kBifMT * kBifRows);
     mbar_init(&sm.mma_idle, 1);
     sm.abort = 0;
     fence_mbar_init();
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     // ------------------------------- TMA producer -------------------------------
     if (lane == 0) {
       uint64_t pol;
-      asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+      asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
       int fills = 0;
       for (int i = 0; i < n_t; ++i) {
         const int s = i % kBifStages;
@@ -254,10 +261,9 @@ __global__ void __launch_bounds__(kBifThreads, 1)
         tma_load_2d(sm.v[s][1], &vmap, 64, y, &sm.v_full[s], pol);
         ++fills;
       }
-      // Every issued copy lands before the CTA moves on (stage s was filled for tiles
-      // s, s + 4, ...; wait for the last phase of each).
+      // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
       for (int s = 0; s < kBifStages && s < fills; ++s) {
-        const int last = (fills - 1 - s) / kBifStages;  // index of the last fill of stage s
+        const int last = (fills - 1 - s) / kBifStages;
         if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr) ||
             !wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr))
           atomicCAS(p.err, 0, kErrBifWait);
@@ -269,44 +275,49 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = f16_idesc(kBifRows, kBifKeys, true, true, false);
       constexpr uint32_t idesc_pv = f16_idesc(kBifRows, kBifD, false, false, true);
-      const uint32_t q_base = smem_addr(sm.q);
-      const uint32_t o_tmem = tmem + 128;
       bool ok = bif_wait(&sm.q_ready, 0, p, abort);
       tc_fence_after();
       for (int i = 0; ok && i <= n_t; ++i) {
         if (i < n_t) {
           const int s = i % kBifStages, b = i & 1;
           ok = bif_wait(&sm.k_full[s], (i / kBifStages) & 1, p, abort);
-          if (ok && i >= 2) ok = bif_wait(&sm.s_free[b], ((i - 2) >> 1) & 1, p, abort);
-          if (!ok) break;
-          tc_fence_after();
           const uint32_t k_base = smem_addr(sm.k[s]);
+          for (int w = 0; ok && w < n_mt; ++w) {
+            if (i >= 2) ok = bif_wait(&sm.s_free[w][b], ((i - 2) >> 1) & 1, p, abort);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t q_base = smem_addr(sm.q[w]);
 #pragma unroll
-          for (int kk = 0; kk < kBifD / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
-            const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
-            const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
-            tc_mma_f16(tmem + b * kBifKeys, a, bd, idesc_qk, kk > 0);
+            for (int kk = 0; kk < kBifD / 16; ++kk) {
+              const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
+              const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
+              const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
+              tc_mma_f16(tmem + w * 128 + b * kBifKeys, a, bd, idesc_qk, kk > 0);
+            }
+            tc_commit(&sm.s_full[w][b]);
           }
+          if (!ok) break;
           tc_commit(&sm.k_empty[s]);
-          tc_commit(&sm.s_full[b]);
         }
         if (i >= 1) {
           const int jj = i - 1, s2 = jj % kBifStages, b2 = jj & 1;
-          ok = bif_wait(&sm.p_full[b2], (jj >> 1) & 1, p, abort);
-          if (ok) ok = bif_wait(&sm.v_conv[s2], (jj / kBifStages) & 1, p, abort);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t p_base = smem_addr(sm.p[b2]);
+          ok = bif_wait(&sm.v_conv[s2], (jj / kBifStages) & 1, p, abort);
           const uint32_t v_base = smem_addr(sm.v[s2]);
+          for (int w = 0; ok && w < n_mt; ++w) {
+            ok = bif_wait(&sm.p_full[w][b2], (jj >> 1) & 1, p, abort);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t p_base = smem_addr(sm.p[w][b2]);
 #pragma unroll
-          for (int kk = 0; kk < kBifKeys / 16; ++kk) {
-            const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
-            tc_mma_f16(o_tmem, a, bd, idesc_pv, jj > 0 || kk > 0);
+            for (int kk = 0; kk < kBifKeys / 16; ++kk) {
+              const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
+              tc_mma_f16(tmem + 256 + w * 128, a, bd, idesc_pv, jj > 0 || kk > 0);
+            }
+            tc_commit(&sm.pv_done[w][b2]);
           }
+          if (!ok) break;
           tc_commit(&sm.v_empty[s2]);
-          tc_commit(&sm.pv_done[b2]);
         }
       }
       // Every issued MMA completes before the tensor memory is released.
@@ -338,10 +349,13 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     }
   } else {
     // ------------------------------- softmax ------------------------------------
-    const int r = tid - 128;                          // row of the M tile = TMEM lane
+    const int w = (warp - 4) >> 2;                    // M tile of this warpgroup
+    const int r = tid - 128 - w * kBifRows;           // row of the M tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + w * 128;
+    const uint32_t o_col = tmem + lane_base + 256 + w * 128;
     const int G = p.n_q_heads / p.n_kv_heads;
-    const int row = mt * kBifRows + r;                // row of this KV head's query matrix
+    const int row = row0 + w * kBifRows + r;          // row of this KV head's query matrix
     const bool valid_row = row < p.rows_per_head;
     {
       const int n = row / G, g = row % G;
@@ -349,112 +363,145 @@ __global__ void __launch_bounds__(kBifThreads, 1)
                                                         (static_cast<int64_t>(n) * p.n_q_heads + h * G + g) * kBifD);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint4 w = valid_row ? src[c] : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sm.q[c >> 3] + sw128_offset(r, c & 7)) = w;
+        const uint4 v = valid_row ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm.q[w][c >> 3] + sw128_offset(r, c & 7)) = v;
       }
       fence_proxy_async_smem();
       mbar_arrive(&sm.q_ready);
     }
+    const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
+    bool ok = w < n_mt;
     for (int i = 0; ok && i < n_t; ++i) {
       const int b = i & 1;
-      ok = bif_wait(&sm.s_full[b], (i >> 1) & 1, p, abort);
+      ok = bif_wait(&sm.s_full[w][b], (i >> 1) & 1, p, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       float x[kBifKeys];
       {
         float t[32];
-        tmem_ld32(tmem + lane_base + b * kBifKeys, t);
+        tmem_ld32(s_col + b * kBifKeys, t);
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c] = t[c];
-        tmem_ld32(tmem + lane_base + b * kBifKeys + 32, t);
+        tmem_ld32(s_col + b * kBifKeys + 32, t);
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[32 + c] = t[c];
         tmem_wait_ld();
       }
       tc_fence_before();
-      mbar_arrive(&sm.s_free[b]);
+      mbar_arrive(&sm.s_free[w][b]);
       const int64_t nvalid = p.prefix_len - (j0 + i) * kBifKeys;
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kBifKeys; ++c) {
-        x[c] = (c < nvalid) ? x[c] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[c]);
-      }
-      const bool need = tmax > m + kBifRescale;
-      const float mn = need ? tmax : m;
-      float rs = 0.f;
       uint32_t ph[kBifKeys / 2];
+      float mn, rs;
+      bool need;
+      if (nvalid >= kBifKeys) {
+        // Full tile: scaled max from the raw extreme, then p = 2^(x s - m) with one FFMA each.
+        float xe = x[0];
+        if (sc >= 0.f) {
 #pragma unroll
-      for (int c = 0; c < kBifKeys; c += 2) {
-        const float p0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn);
-        const float p1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn);
-        rs += p0 + p1;
-        const __half2 hv = __floats2half2_rn(p0, p1);
-        ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int c = 1; c < kBifKeys; ++c) xe = fmaxf(xe, x[c]);
+        } else {
+#pragma unroll
+          for (int c = 1; c < kBifKeys; ++c) xe = fminf(xe, x[c]);
+        }
+        const float tmax = xe * sc;
+        need = tmax > m + kBifRescale;
+        mn = need ? tmax : m;
+        const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kBifKeys; c += 2) {
+          const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), s2, nm);
+          const float2 pp = make_float2(ex2(y.x), ex2(y.y));
+          acc = __fadd2_rn(acc, pp);
+          const __half2 hv = __floats2half2_rn(pp.x, pp.y);
+          ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        rs = acc.x + acc.y;
+      } else {
+        // Last, partial tile of the context: keys past its end get p = 0.
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kBifKeys; ++c) {
+          x[c] = (c < nvalid) ? x[c] * sc : -INFINITY;
+          tmax = fmaxf(tmax, x[c]);
+        }
+        need = tmax > m + kBifRescale;
+        mn = need ? tmax : m;
+        rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < kBifKeys; c += 2) {
+          const float p0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn);
+          const float p1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn);
+          rs += p0 + p1;
+          const __half2 hv = __floats2half2_rn(p0, p1);
+          ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
       }
       // P buffer b was last read by the P V product of tile i - 2.
-      if (i >= 2) ok = bif_wait(&sm.pv_done[b], ((i - 2) >> 1) & 1, p, abort);
+      if (i >= 2) ok = bif_wait(&sm.pv_done[w][b], ((i - 2) >> 1) & 1, p, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(sm.p[b] + sw128_offset(r, c)) =
+        *reinterpret_cast<uint4*>(sm.p[w][b] + sw128_offset(r, c)) =
             make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
       fence_proxy_async_smem();
       const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
       // O holds tiles 0..i-1: rescale it (after the P V product of tile i-1) when m grew.
       if (__any_sync(0xffffffffu, need && i >= 1)) {
-        ok = bif_wait(&sm.pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, p, abort);
+        ok = bif_wait(&sm.pv_done[w][(i - 1) & 1], ((i - 1) >> 1) & 1, p, abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int q4 = 0; q4 < kBifD / 32; ++q4) {
           float o[32];
-          tmem_ld32(tmem + lane_base + 128 + q4 * 32, o);
+          tmem_ld32(o_col + q4 * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] *= alpha;
-          tmem_st32(tmem + lane_base + 128 + q4 * 32, o);
+          tmem_st32(o_col + q4 * 32, o);
         }
         tmem_wait_st();
       }
       l = l * alpha + rs;
       m = mn;
       tc_fence_before();
-      mbar_arrive(&sm.p_full[b]);
+      mbar_arrive(&sm.p_full[w][b]);
     }
     // The chunk's statistics of this row.
-    float* dst = p.part + ((static_cast<int64_t>(chunk) * p.n_kv_heads + h) * p.rows_per_head + row) * kBifPartRow;
-    if (n_t > 0 && ok) {
-      ok = bif_wait(&sm.pv_done[(n_t - 1) & 1], ((n_t - 1) >> 1) & 1, p, abort);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (n_t > 0 && ok) {
-      tc_fence_after();
+    if (w < n_mt) {
+      float* dst =
+          p.part + ((static_cast<int64_t>(chunk) * p.n_kv_heads + h) * p.rows_per_head + row) * kBifPartRow;
+      if (n_t > 0 && ok) {
+        ok = bif_wait(&sm.pv_done[w][(n_t - 1) & 1], ((n_t - 1) >> 1) & 1, p, abort);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      if (n_t > 0 && ok) {
+        tc_fence_after();
 #pragma unroll
-      for (int q4 = 0; q4 < kBifD / 32; ++q4) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + 128 + q4 * 32, o);
-        tmem_wait_ld();
-        if (valid_row) {
+        for (int q4 = 0; q4 < kBifD / 32; ++q4) {
+          float o[32];
+          tmem_ld32(o_col + q4 * 32, o);
+          tmem_wait_ld();
+          if (valid_row) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(dst + 4 + q4 * 32 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + 4 + q4 * 32 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          }
         }
+        if (valid_row) {
+          dst[0] = m;
+          dst[1] = l;
+        }
+      } else if (valid_row) {
+        // Empty chunk, or an aborted one (the error word is set and the merge writes NaN).
+        dst[0] = -INFINITY;
+        dst[1] = 0.f;
+        for (int c = 0; c < kBifD; ++c) dst[4 + c] = 0.f;
       }
-      if (valid_row) {
-        dst[0] = m;
-        dst[1] = l;
-      }
-    } else if (valid_row) {
-      // Empty chunk, or an aborted one (the error word is set and the merge writes NaN).
-      dst[0] = -INFINITY;
-      dst[1] = 0.f;
-      for (int c = 0; c < kBifD; ++c) dst[4 + c] = 0.f;
     }
   }
   tc_fence_before();
@@ -470,45 +517,65 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 // ---------------------------------------------------------------------------------------------
 
 // Suffix part given normalised (out_s, lse_s); it enters as m = lse_s log2(e), l = 1, o = out_s.
+// One thread per 4 columns of an output row; the chunk loops are unrolled so that the
+// partials' loads are in flight together.
 __global__ void merge_prefix_suffix_kernel(const float* __restrict__ part, int n_chunks, int n_kv_heads,
                                            int rows_per_head, const float* __restrict__ out_s,
                                            const float* __restrict__ lse_s, float* __restrict__ out,
                                            float* __restrict__ lse, int n_samples, int n_q_heads,
                                            const int* __restrict__ err) {
+  constexpr int Q = kBifD / 4;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(n_samples) * n_q_heads * kBifD;
+  const int64_t total = static_cast<int64_t>(n_samples) * n_q_heads * Q;
   if (i >= total) return;
-  const int d = static_cast<int>(i % kBifD);
-  const int64_t rq = i / kBifD;  // n * Hq + hq
+  const int d4 = static_cast<int>(i % Q) * 4;
+  const int64_t rq = i / Q;  // n * Hq + hq
   const int n = static_cast<int>(rq / n_q_heads), hq = static_cast<int>(rq % n_q_heads);
   const int G = n_q_heads / n_kv_heads;
   const int h = hq / G, g = hq % G;
-  const int64_t prow = static_cast<int64_t>(h) * rows_per_head + n * G + g;
+  const float* base = part + (static_cast<int64_t>(h) * rows_per_head + n * G + g) * kBifPartRow;
   const int64_t stride = static_cast<int64_t>(n_kv_heads) * rows_per_head * kBifPartRow;
   const float ls = lse_s[rq];
   const float ms = (ls == -INFINITY) ? -INFINITY : ls * 1.44269504088896340736f;
   float M = ms;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, part[c * stride + prow * kBifPartRow]);
-  float L = 0.f, O = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, base[c * stride]);
+  float L = 0.f;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
   if (M != -INFINITY) {
+#pragma unroll 8
     for (int c = 0; c < n_chunks; ++c) {
-      const float* pc = part + c * stride + prow * kBifPartRow;
-      const float w = (pc[0] == -INFINITY) ? 0.f : ex2(pc[0] - M);
-      L += w * pc[1];
-      O += w * pc[4 + d];
+      const float* pc = base + c * stride;
+      const float2 ml = *reinterpret_cast<const float2*>(pc);
+      const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
+      const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
+      L += w * ml.y;
+      O.x += w * o.x;
+      O.y += w * o.y;
+      O.z += w * o.z;
+      O.w += w * o.w;
     }
     const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+    const float4 os = *reinterpret_cast<const float4*>(out_s + rq * kBifD + d4);
     L += w;
-    O += w * out_s[rq * kBifD + d];
+    O.x += w * os.x;
+    O.y += w * os.y;
+    O.z += w * os.z;
+    O.w += w * os.w;
   }
-  float ov = 0.f, lv = -INFINITY;
+  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lv = -INFINITY;
   if (L > 0.f) {
-    ov = O / L;
+    ov = make_float4(O.x / L, O.y / L, O.z / L, O.w / L);
     lv = (M + log2f(L)) * 0.693147180559945309f;
   }
-  if (*reinterpret_cast<const volatile int*>(err) != 0 || ls != ls) ov = lv = __int_as_float(0x7fc00000);
-  out[rq * kBifD + d] = ov;
-  if (d == 0) lse[rq] = lv;
+  if (*reinterpret_cast<const volatile int*>(err) != 0 || ls != ls) {
+    const float nan = __int_as_float(0x7fc00000);
+    ov = make_float4(nan, nan, nan, nan);
+    lv = nan;
+  }
+  *reinterpret_cast<float4*>(out + rq * kBifD + d4) = ov;
+  if (d4 == 0) lse[rq] = lv;
 }
 
 }  // namespace ta

@@ -62,52 +62,64 @@ struct SplitParams {
   int32_t n_tiles[kMaxSeqPerLaunch];       // tiles per (sequence, KV head), >= 1
 };
 
-// Build-time tuning of the split kernel (defaults measured best on B200; see the design notes).
+// Tile configurations of the split kernel (measured on B200; see the design notes).
+// LongTiles: 12 consumer warps, 8 row elements per lane, 48 KB K and V tiles, a 2-deep ring:
+// long sequences stream at the HBM roofline.  ShortTiles: 8 warps, 16 elements per lane,
+// 16 KB tiles (64 tokens at D = 128), a 4-deep ring: short sequences waste less of their
+// last tile and pay less per (sequence, KV head) boundary.
 #ifndef TA_SPLIT_WARPS
-#define TA_SPLIT_WARPS 12  // consumer warps per CTA
+#define TA_SPLIT_WARPS 12
 #endif
 #ifndef TA_SPLIT_STAGES
-#define TA_SPLIT_STAGES 2  // depth of the shared-memory ring
+#define TA_SPLIT_STAGES 2
 #endif
 #ifndef TA_SPLIT_ELEMS
-#define TA_SPLIT_ELEMS 8  // row elements per lane when G <= 4 (G = 8 uses half, at least one chunk)
+#define TA_SPLIT_ELEMS 8
+#endif
+#ifndef TA_SPLIT_TILE_BYTES
+#define TA_SPLIT_TILE_BYTES 49152
 #endif
 #ifndef TA_SPLIT_KV_BARRIERS
 #define TA_SPLIT_KV_BARRIERS 0  // 1: separate "K landed" and "V landed" barriers per stage
 #endif
-#ifndef TA_SPLIT_TILE_BYTES
-#define TA_SPLIT_TILE_BYTES 49152  // target bytes of one K (or V) tile
-#endif
+
+struct LongTiles {
+  static constexpr int warps = TA_SPLIT_WARPS, stages = TA_SPLIT_STAGES, elems = TA_SPLIT_ELEMS,
+                       tile_bytes = TA_SPLIT_TILE_BYTES;
+};
+struct ShortTiles {
+  static constexpr int warps = 8, stages = 4, elems = 16, tile_bytes = 16384;
+};
 
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100 (227 KB)
 
-// G = 8 keeps 8 consumer warps: its q and o registers need more than the 128 per thread
-// that 13 resident warps leave (4 warps on one SM sub-partition).
-template <typename T, int D_, int G_, int NCW_ = (G_ >= 8 ? 8 : TA_SPLIT_WARPS), int NSTAGE_ = TA_SPLIT_STAGES>
+template <typename T, int D_, int G_, class V = LongTiles>
 struct SplitCfg {
   static constexpr int D = D_;
   static constexpr int G = G_;
   static constexpr int ELEM = sizeof(T);
   static constexpr int EPC = 16 / ELEM;        // elements per 16-byte chunk
   // Row elements held by one lane (at least one chunk; G = 8 halves it to bound registers).
-  static constexpr int E = (G >= 8) ? (TA_SPLIT_ELEMS / 2 > EPC ? TA_SPLIT_ELEMS / 2 : EPC) : TA_SPLIT_ELEMS;
+  static constexpr int E = (G >= 8) ? (V::elems / 2 > EPC ? V::elems / 2 : EPC) : V::elems;
   static constexpr int E2 = E / 2;             // ... as float pairs (packed FP32 math)
   static constexpr int LPT = D / E;            // lanes per token
   static constexpr int TPW = 32 / LPT;         // tokens per warp step
   static constexpr int ROW = D * ELEM;         // bytes per token row
-  static constexpr int NCW = NCW_;             // consumer warps
-  static constexpr int NSTAGE = NSTAGE_;
+  // G = 8 keeps at most 8 consumer warps: its q and o registers need more than the 128 per
+  // thread that 13 resident warps leave (4 warps on one SM sub-partition).
+  static constexpr int NCW = (G >= 8 && V::warps > 8) ? 8 : V::warps;  // consumer warps
+  static constexpr int NSTAGE = V::stages;
   static constexpr int MERGE_BATCH = 128;      // partials whose weights are staged at once
   // Shared memory besides the ring: per-warp statistics, merge weights, barriers and flags.
   static constexpr int FIXED_SMEM = NCW * G * D * 4 + 2 * NCW * G * 4 + MERGE_BATCH * G * 4 + 1024;
   static constexpr int MAX_TILE_BYTES = (kSmemLimit - FIXED_SMEM) / (2 * NSTAGE);
-  static constexpr int TILE_TARGET = TA_SPLIT_TILE_BYTES < MAX_TILE_BYTES ? TA_SPLIT_TILE_BYTES : MAX_TILE_BYTES;
+  static constexpr int TILE_TARGET = V::tile_bytes < MAX_TILE_BYTES ? V::tile_bytes : MAX_TILE_BYTES;
   static constexpr int STEPS_FIT = TILE_TARGET / (ROW * NCW * TPW);
   // Tokens per warp per tile (phase length).  Longer phases give more independent work per
   // warp but hold more registers: 8 (4 when G = 8, whose q and o take twice the registers).
   static constexpr int MAX_STEPS = G >= 8 ? 4 : 8;
   static constexpr int STEPS = STEPS_FIT < 1 ? 1 : (STEPS_FIT > MAX_STEPS ? MAX_STEPS : STEPS_FIT);
-  static constexpr int TILE = NCW * STEPS * TPW;  // tokens per tile (about 16 KB of K and of V)
+  static constexpr int TILE = NCW * STEPS * TPW;  // tokens per tile
   static constexpr int PPC = EPC / 2;          // float pairs per chunk
   static constexpr int NCH = E / EPC;          // chunks per lane per row
   static constexpr int TILE_BYTES = TILE * ROW;
@@ -336,10 +348,10 @@ __device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq,
 // The kernel
 // ---------------------------------------------------------------------------------------------
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(SplitCfg<T, D, G>::THREADS, 1)
+template <typename T, int D, int G, class V>
+__global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
     split_kv_decode_kernel(const __grid_constant__ SplitParams p) {
-  using C = SplitCfg<T, D, G>;
+  using C = SplitCfg<T, D, G, V>;
   constexpr int E2 = C::E2;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   SplitSmem<C>& sm = *reinterpret_cast<SplitSmem<C>*>(smem_raw);

@@ -40,32 +40,47 @@ struct KernelInfo {
   int threads;
 };
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, class V>
 KernelInfo make_info() {
-  using C = SplitCfg<T, D, G>;
-  return KernelInfo{&split_kv_decode_kernel<T, D, G>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
+  using C = SplitCfg<T, D, G, V>;
+  return KernelInfo{&split_kv_decode_kernel<T, D, G, V>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
 }
 
-template <typename T, int D>
+template <typename T, int D, class V>
 bool pick_g(int G, KernelInfo* ki) {
   switch (G) {
-    case 1: *ki = make_info<T, D, 1>(); return true;
-    case 2: *ki = make_info<T, D, 2>(); return true;
-    case 4: *ki = make_info<T, D, 4>(); return true;
-    case 8: *ki = make_info<T, D, 8>(); return true;
+    case 1: *ki = make_info<T, D, 1, V>(); return true;
+    case 2: *ki = make_info<T, D, 2, V>(); return true;
+    case 4: *ki = make_info<T, D, 4, V>(); return true;
+    case 8: *ki = make_info<T, D, 8, V>(); return true;
     default: return false;
   }
 }
 
-bool pick_kernel(ta_dtype dt, int D, int G, KernelInfo* ki) {
+template <class V>
+bool pick_variant(ta_dtype dt, int D, int G, KernelInfo* ki) {
   if (dt == TA_BF16) {
-    if (D == 64) return pick_g<__nv_bfloat16, 64>(G, ki);
-    if (D == 128) return pick_g<__nv_bfloat16, 128>(G, ki);
+    if (D == 64) return pick_g<__nv_bfloat16, 64, V>(G, ki);
+    if (D == 128) return pick_g<__nv_bfloat16, 128, V>(G, ki);
   } else if (dt == TA_F32) {
-    if (D == 64) return pick_g<float, 64>(G, ki);
-    if (D == 128) return pick_g<float, 128>(G, ki);
+    if (D == 64) return pick_g<float, 64, V>(G, ki);
+    if (D == 128) return pick_g<float, 128, V>(G, ki);
   }
   return false;
+}
+
+bool pick_kernel(ta_dtype dt, int D, int G, bool short_tiles, KernelInfo* ki) {
+  return short_tiles ? pick_variant<ShortTiles>(dt, D, G, ki) : pick_variant<LongTiles>(dt, D, G, ki);
+}
+
+// Tile configuration for a batch: short tiles when the mean (sequence, KV head) unit is
+// shorter than 1024 tokens, unless the options force one.
+bool use_short_tiles(const int64_t* seqlens, int batch, const ta_options* opts) {
+  if (opts && opts->split_tiles == 1) return false;
+  if (opts && opts->split_tiles == 2) return true;
+  int64_t total = 0;
+  for (int b = 0; b < batch; ++b) total += seqlens[b];
+  return batch > 0 && total < 1024LL * batch;
 }
 
 // Resident CTAs of an instance on the current device (sets the shared-memory opt-in once).
@@ -171,7 +186,8 @@ ta_status check_opts(const ta_options* o) {
   if (!o) return TA_OK;
   if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1) return TA_ERR_INVALID_ARG;
   if (o->prefix_path < 0 || o->prefix_path > 2) return TA_ERR_INVALID_ARG;
-  for (int i = 0; i < 4; ++i)
+  if (o->split_tiles < 0 || o->split_tiles > 2) return TA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
     if (o->reserved[i] != 0) return TA_ERR_INVALID_ARG;
   return TA_OK;
 }
@@ -183,7 +199,7 @@ ta_status check_shape(const int64_t* seqlens, int batch, int Hq, int Hkv, int D,
   for (int b = 0; b < batch; ++b)
     if (seqlens[b] < 0) return TA_ERR_INVALID_ARG;
   if (dt != TA_BF16 && dt != TA_F32) return TA_ERR_INVALID_ARG;
-  if (!pick_kernel(dt, D, Hq / Hkv, ki)) return TA_ERR_UNSUPPORTED;
+  if (!pick_kernel(dt, D, Hq / Hkv, false, ki)) return TA_ERR_UNSUPPORTED;
   return TA_OK;
 }
 
@@ -262,6 +278,7 @@ ta_status validate(const DecodeArgs& a, const ta_options* opts, bool check_point
   s = check_shape(a.seqlens, a.batch, a.Hq, a.Hkv, a.D, a.dt, ki);
   if (s != TA_OK) return s;
   if (!std::isfinite(a.scale)) return TA_ERR_INVALID_ARG;
+  pick_kernel(a.dt, a.D, a.Hq / a.Hkv, use_short_tiles(a.seqlens, a.batch, opts), ki);
   if (check_pointers && a.batch > 0)
     return check_ptrs(a.q, a.k, a.v, a.out, a.lse, any_tokens(a.seqlens, a.batch));
   return TA_OK;
@@ -352,7 +369,7 @@ struct BifArgs {
 };
 
 struct BifPlan {
-  KernelInfo ki;
+  KernelInfo ki, ki_suffix;  // split kernel of the prefix pass (per sample) and of the suffix pass
   Plan prefix, suffix;
   std::vector<int64_t> prefix_lens, prefix_offs;
   size_t scratch_off = 0, body_off = 0, suffix_off = 0, total = 0;
@@ -427,15 +444,20 @@ ta_status bif_validate(const BifArgs& a, const ta_options* opts, bool check_poin
 }
 
 ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& ki, BifPlan* bp) {
-  bp->ki = ki;
   bp->prefix_lens.assign(a.N, a.P);
   bp->prefix_offs.assign(a.N, 0);
+  bp->ki = ki;
+  bp->ki_suffix = ki;
+  if (a.N > 0) {
+    pick_kernel(TA_BF16, a.D, a.Hq / a.Hkv, use_short_tiles(bp->prefix_lens.data(), a.N, opts), &bp->ki);
+    pick_kernel(TA_BF16, a.D, a.Hq / a.Hkv, use_short_tiles(a.suffix_lens, a.N, opts), &bp->ki_suffix);
+  }
   DecodeArgs pre{TA_BF16, a.q, a.kp, a.vp, bp->prefix_lens.data(), bp->prefix_offs.data(), a.N, a.Hq, a.Hkv, a.D,
                  a.scale, a.out, a.lse};
-  ta_status s = plan_for(pre, opts, ki, &bp->prefix);
+  ta_status s = plan_for(pre, opts, bp->ki, &bp->prefix);
   if (s != TA_OK) return s;
   DecodeArgs suf{TA_BF16, a.q, a.ks, a.vs, a.suffix_lens, nullptr, a.N, a.Hq, a.Hkv, a.D, a.scale, a.out, a.lse};
-  s = plan_for(suf, opts, ki, &bp->suffix);
+  s = plan_for(suf, opts, bp->ki_suffix, &bp->suffix);
   if (s != TA_OK) return s;
   const size_t rows = static_cast<size_t>(a.N) * a.Hq;
   bp->scratch_off = kHeaderBytes;
@@ -454,7 +476,7 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
     if (s != TA_OK) return s;
     bp->tc = true;
     bp->rows_per_head = a.N * (a.Hq / a.Hkv);
-    bp->mtiles = (bp->rows_per_head + kBifRows - 1) / kBifRows;
+    bp->mtiles = (bp->rows_per_head + kBifMT * kBifRows - 1) / (kBifMT * kBifRows);  // CTAs per (chunk, head)
     const int64_t tiles = (a.P + kBifKeys - 1) / kBifKeys;
     int64_t chunks = sms / (static_cast<int64_t>(bp->mtiles) * a.Hkv);
     chunks = std::max<int64_t>(1, std::min<int64_t>(chunks, tiles));
@@ -499,10 +521,10 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
       bif_prefix_kernel<<<grid, kBifThreads, sizeof(BifSmem) + 1024, st>>>(kmap, vmap, bpp);
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return cuda_fail(e);
-      s = launch_plan(bp.suffix, bp.ki, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
+      s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                       base + bp.suffix_off, err, st);
       if (s != TA_OK) return s;
-      const int64_t n = static_cast<int64_t>(rows) * a.D;
+      const int64_t n = static_cast<int64_t>(rows) * (kBifD / 4);  // one thread per 4 columns of a row
       merge_prefix_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
           bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse, a.N, a.Hq, err);
       e = cudaGetLastError();
@@ -514,7 +536,7 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
   s = launch_plan(bp.prefix, bp.ki, a.q, a.kp, a.vp, out_p, lse_p, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                   base + bp.body_off, err, st);
   if (s != TA_OK) return s;
-  s = launch_plan(bp.suffix, bp.ki, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
+  s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                   base + bp.suffix_off, err, st);
   if (s != TA_OK) return s;
   const int64_t n = static_cast<int64_t>(rows) * a.D;

@@ -82,7 +82,9 @@ typedef struct {
   int32_t prefix_path;     /* bifurcated calls only.  0: automatic (tensor-core prefix pass when
                               head_dim is 128 and the prefix is not empty); 1: tensor-core pass
                               (TA_ERR_UNSUPPORTED if not possible); 2: split-KV pass per sample */
-  int32_t reserved[4];     /* must be 0 */
+  int32_t split_tiles;     /* split-KV tile configuration.  0: automatic (short tiles when the mean
+                              sequence is under 1024 tokens); 1: long tiles; 2: short tiles */
+  int32_t reserved[3];     /* must be 0 */
 } ta_options;
 
 /* A short English name of a status code (static storage). */

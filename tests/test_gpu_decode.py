@@ -28,26 +28,30 @@ def oracle_of(inp, sp, pairs=None):
 RAGGED = [1, 0, 31, 33, 64, 65, 127, 129, 1000, 3001]
 
 
+@pytest.mark.parametrize("tiles", [1, 2])  # long and short tile configurations
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-def test_every_instance_ragged(dtype, D, G):
+def test_every_instance_ragged(dtype, D, G, tiles):
+    import exact_long_context_split_b200 as ta
+
     Hkv = 2
     sp = spec(RAGGED, G * Hkv, Hkv, D, dtype=dtype, seed=100 + G + D)
     inp = synth.make_decode_inputs(sp)
-    out, lse = decode_gpu(inp, sp)
+    out, lse = decode_gpu(inp, sp, ta.make_options(split_tiles=tiles))
     ref_out, ref_lse = oracle_of(inp, sp)
     compare(out, lse, ref_out, ref_lse)
 
 
+@pytest.mark.parametrize("tiles", [1, 2])
 @pytest.mark.parametrize("num_ctas", [1, 2, 7, 37, 148, 1000, 100000])
-def test_grid_sizes_and_merge_trees(num_ctas):
+def test_grid_sizes_and_merge_trees(num_ctas, tiles):
     """From one CTA doing every tile (no merge) to one tile per CTA (deep merge trees)."""
     sp = spec([5000, 77, 0, 2100], 16, 4, 128, seed=5)
     inp = synth.make_decode_inputs(sp)
     import exact_long_context_split_b200 as ta
 
-    opts = ta.make_options(num_ctas=num_ctas)
+    opts = ta.make_options(num_ctas=num_ctas, split_tiles=tiles)
     out, lse = decode_gpu(inp, sp, opts)
     ref_out, ref_lse = oracle_of(inp, sp)
     compare(out, lse, ref_out, ref_lse)
