@@ -15,7 +15,8 @@
 //
 // One CTA owns up to 256 rows (two M tiles of 128) and a contiguous chunk of 64-key
 // tiles of the context; both M tiles consume every K/V tile it loads.
-// Roles (12 warps):  warp 0 lane 0: TMA producer of K and V tiles;  warp 1: TMEM
+// Roles (13 warps):  warp 0 lane 0 / warp 12 lane 0: TMA producers of the K and of the V
+// tiles (K stages free as soon as QK is done, V stages only after P V);  warp 1: TMEM
 // allocation and lane 0 issues tcgen05.mma;  warps 2-3: convert each V tile from bf16
 // to fp16 in place (P is kept in fp16 for the P V product: bf16 P is too coarse);
 // warps 4-7 and 8-11: softmax of M tile 0 and 1, thread t owns row t = TMEM lane t.
@@ -37,7 +38,7 @@ constexpr int kBifMT = 2;           // M tiles per CTA: the CTA's 256 rows share
 constexpr int kBifKeys = 64;        // keys per tile (N of S, K of P V)
 constexpr int kBifD = 128;          // head_dim
 constexpr int kBifStages = 3;       // K ring and V ring depth
-constexpr int kBifThreads = 384;    // 12 warps
+constexpr int kBifThreads = 416;    // 13 warps
 constexpr int kBifTmemCols = 512;   // S: 2 tiles x 2 buffers x 64 columns; O: 2 tiles x 128 columns
 constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
 
@@ -239,34 +240,32 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 0) {
-    // ------------------------------- TMA producer -------------------------------
+  if (warp == 0 || warp == 12) {
+    // ------------------------------- TMA producers ------------------------------
+    // warp 0 streams K, warp 12 streams V; each refills a stage once its own product freed it.
     if (lane == 0) {
+      const bool is_k = warp == 0;
+      uint64_t* full = is_k ? sm.k_full : sm.v_full;
+      uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
+      const CUtensorMap* map = is_k ? &kmap : &vmap;
       uint64_t pol;
       asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
       int fills = 0;
       for (int i = 0; i < n_t; ++i) {
         const int s = i % kBifStages;
-        if (i >= kBifStages) {
-          const uint32_t par = ((i / kBifStages) - 1) & 1;
-          if (!bif_wait(&sm.k_empty[s], par, p, abort) || !bif_wait(&sm.v_empty[s], par, p, abort)) break;
-        }
+        if (i >= kBifStages && !bif_wait(&empty[s], ((i / kBifStages) - 1) & 1, p, abort)) break;
         if (*abort) break;
         const int y = static_cast<int>(h * p.prefix_len + (j0 + i) * kBifKeys);
-        mbar_arrive_expect_tx(&sm.k_full[s], 2 * kBifKeys * 128);
-        tma_load_2d(sm.k[s][0], &kmap, 0, y, &sm.k_full[s], pol);
-        tma_load_2d(sm.k[s][1], &kmap, 64, y, &sm.k_full[s], pol);
-        mbar_arrive_expect_tx(&sm.v_full[s], 2 * kBifKeys * 128);
-        tma_load_2d(sm.v[s][0], &vmap, 0, y, &sm.v_full[s], pol);
-        tma_load_2d(sm.v[s][1], &vmap, 64, y, &sm.v_full[s], pol);
+        uint8_t* dst = is_k ? sm.k[s][0] : sm.v[s][0];
+        mbar_arrive_expect_tx(&full[s], 2 * kBifKeys * 128);
+        tma_load_2d(dst, map, 0, y, &full[s], pol);
+        tma_load_2d(dst + kBifKeys * 128, map, 64, y, &full[s], pol);
         ++fills;
       }
       // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
       for (int s = 0; s < kBifStages && s < fills; ++s) {
         const int last = (fills - 1 - s) / kBifStages;
-        if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr) ||
-            !wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr))
-          atomicCAS(p.err, 0, kErrBifWait);
+        if (!wait_phase(&full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
       }
     }
     __syncwarp();
@@ -277,47 +276,84 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       constexpr uint32_t idesc_pv = f16_idesc(kBifRows, kBifD, false, false, true);
       bool ok = bif_wait(&sm.q_ready, 0, p, abort);
       tc_fence_after();
-      for (int i = 0; ok && i <= n_t; ++i) {
-        if (i < n_t) {
-          const int s = i % kBifStages, b = i & 1;
-          ok = bif_wait(&sm.k_full[s], (i / kBifStages) & 1, p, abort);
-          const uint32_t k_base = smem_addr(sm.k[s]);
-          for (int w = 0; ok && w < n_mt; ++w) {
-            if (i >= 2) ok = bif_wait(&sm.s_free[w][b], ((i - 2) >> 1) & 1, p, abort);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t q_base = smem_addr(sm.q[w]);
+      // S = Q K^T of tile t into S buffer t & 1 of every active M tile.
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t % kBifStages, b = t & 1;
+        if (!bif_wait(&sm.k_full[s], (t / kBifStages) & 1, p, abort)) return false;
+        const uint32_t k_base = smem_addr(sm.k[s]);
+        for (int w = 0; w < n_mt; ++w) {
+          // Buffer b last held tile t - 2; its softmax has loaded it once s_free fires.
+          if (t >= 2 && !bif_wait(&sm.s_free[w][b], ((t - 2) >> 1) & 1, p, abort)) return false;
+          tc_fence_after();
+          const uint32_t q_base = smem_addr(sm.q[w]);
 #pragma unroll
-            for (int kk = 0; kk < kBifD / 16; ++kk) {
-              const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
-              const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
-              const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
-              tc_mma_f16(tmem + w * 128 + b * kBifKeys, a, bd, idesc_qk, kk > 0);
-            }
-            tc_commit(&sm.s_full[w][b]);
+          for (int kk = 0; kk < kBifD / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
+            const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
+            const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
+            tc_mma_f16(tmem + w * 128 + b * kBifKeys, a, bd, idesc_qk, kk > 0);
           }
-          if (!ok) break;
-          tc_commit(&sm.k_empty[s]);
+          tc_commit(&sm.s_full[w][b]);
         }
-        if (i >= 1) {
-          const int jj = i - 1, s2 = jj % kBifStages, b2 = jj & 1;
-          ok = bif_wait(&sm.v_conv[s2], (jj / kBifStages) & 1, p, abort);
-          const uint32_t v_base = smem_addr(sm.v[s2]);
-          for (int w = 0; ok && w < n_mt; ++w) {
-            ok = bif_wait(&sm.p_full[w][b2], (jj >> 1) & 1, p, abort);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t p_base = smem_addr(sm.p[w][b2]);
+        tc_commit(&sm.k_empty[s]);
+        return true;
+      };
+      // O += P V of tile t for every active M tile.
+      auto issue_pv = [&](int t) -> bool {
+        const int s = t % kBifStages, b = t & 1;
+        if (!bif_wait(&sm.v_conv[s], (t / kBifStages) & 1, p, abort)) return false;
+        const uint32_t v_base = smem_addr(sm.v[s]);
+        for (int w = 0; w < n_mt; ++w) {
+          if (!bif_wait(&sm.p_full[w][b], (t >> 1) & 1, p, abort)) return false;
+          tc_fence_after();
+          const uint32_t p_base = smem_addr(sm.p[w][b]);
 #pragma unroll
-            for (int kk = 0; kk < kBifKeys / 16; ++kk) {
-              const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
-              const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
-              tc_mma_f16(tmem + 256 + w * 128, a, bd, idesc_pv, jj > 0 || kk > 0);
-            }
-            tc_commit(&sm.pv_done[w][b2]);
+          for (int kk = 0; kk < kBifKeys / 16; ++kk) {
+            const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
+            tc_mma_f16(tmem + 256 + w * 128, a, bd, idesc_pv, t > 0 || kk > 0);
           }
-          if (!ok) break;
-          tc_commit(&sm.v_empty[s2]);
+          tc_commit(&sm.pv_done[w][b]);
+        }
+        tc_commit(&sm.v_empty[s]);
+        return true;
+      };
+      // Two streams, QK(tq) and PV(tp), each in tile order; whichever has its inputs ready
+      // is issued, so neither waits for the other (the tensor pipe runs them in issue order).
+      // QK(t) needs K(t) and the softmax of t - 2 to have loaded its S buffer; PV(t) needs
+      // V(t) converted and P(t) written.
+      auto qk_ready = [&](int t) {
+        if (!mbar_test_wait(&sm.k_full[t % kBifStages], (t / kBifStages) & 1)) return false;
+        for (int w = 0; t >= 2 && w < n_mt; ++w)
+          if (!mbar_test_wait(&sm.s_free[w][t & 1], ((t - 2) >> 1) & 1)) return false;
+        return true;
+      };
+      auto pv_ready = [&](int t) {
+        if (!mbar_test_wait(&sm.v_conv[t % kBifStages], (t / kBifStages) & 1)) return false;
+        for (int w = 0; w < n_mt; ++w)
+          if (!mbar_test_wait(&sm.p_full[w][t & 1], (t >> 1) & 1)) return false;
+        return true;
+      };
+      int tq = 0, tp = 0;
+      uint64_t t_idle = global_timer_ns();
+      while (ok && tp < n_t) {
+        bool progress = false;
+        if (tq < n_t && qk_ready(tq)) {
+          ok = issue_qk(tq++);
+          progress = true;
+        }
+        if (ok && tp < tq && pv_ready(tp)) {
+          ok = issue_pv(tp++);
+          progress = true;
+        }
+        if (progress) {
+          t_idle = global_timer_ns();
+        } else if (*abort) {
+          ok = false;
+        } else if (static_cast<int64_t>(global_timer_ns() - t_idle) > p.wait_limit_ns) {
+          atomicCAS(p.err, 0, kErrBifWait);
+          *abort = 1;
+          ok = false;
         }
       }
       // Every issued MMA completes before the tensor memory is released.
@@ -397,28 +433,41 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       bool need;
       if (nvalid >= kBifKeys) {
         // Full tile: scaled max from the raw extreme, then p = 2^(x s - m) with one FFMA each.
-        float xe = x[0];
+        // Extreme of the raw scores in 8 independent chains, then a tree.
+        float xe[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xe[k] = x[k];
         if (sc >= 0.f) {
 #pragma unroll
-          for (int c = 1; c < kBifKeys; ++c) xe = fmaxf(xe, x[c]);
+          for (int c = 8; c < kBifKeys; ++c) xe[c & 7] = fmaxf(xe[c & 7], x[c]);
+#pragma unroll
+          for (int k = 4; k >= 1; k >>= 1)
+#pragma unroll
+            for (int j = 0; j < k; ++j) xe[j] = fmaxf(xe[j], xe[j + k]);
         } else {
 #pragma unroll
-          for (int c = 1; c < kBifKeys; ++c) xe = fminf(xe, x[c]);
+          for (int c = 8; c < kBifKeys; ++c) xe[c & 7] = fminf(xe[c & 7], x[c]);
+#pragma unroll
+          for (int k = 4; k >= 1; k >>= 1)
+#pragma unroll
+            for (int j = 0; j < k; ++j) xe[j] = fminf(xe[j], xe[j + k]);
         }
-        const float tmax = xe * sc;
+        const float tmax = xe[0] * sc;
         need = tmax > m + kBifRescale;
         mn = need ? tmax : m;
         const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
-        float2 acc = make_float2(0.f, 0.f);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < kBifKeys; c += 2) {
           const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), s2, nm);
           const float2 pp = make_float2(ex2(y.x), ex2(y.y));
-          acc = __fadd2_rn(acc, pp);
+          acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], pp);
           const __half2 hv = __floats2half2_rn(pp.x, pp.y);
           ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
         }
-        rs = acc.x + acc.y;
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+        const float2 a = __fadd2_rn(a01, a23);
+        rs = a.x + a.y;
       } else {
         // Last, partial tile of the context: keys past its end get p = 0.
         float tmax = -INFINITY;

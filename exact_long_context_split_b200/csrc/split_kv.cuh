@@ -64,9 +64,9 @@ struct SplitParams {
 
 // Tile configurations of the split kernel (measured on B200; see the design notes).
 // LongTiles: 12 consumer warps, 8 row elements per lane, 48 KB K and V tiles, a 2-deep ring:
-// long sequences stream at the HBM roofline.  ShortTiles: 8 warps, 16 elements per lane,
+// long sequences stream at the HBM roofline.  ShortTiles: 8 warps, 8 elements per lane,
 // 16 KB tiles (64 tokens at D = 128), a 4-deep ring: short sequences waste less of their
-// last tile and pay less per (sequence, KV head) boundary.
+// last tile.
 #ifndef TA_SPLIT_WARPS
 #define TA_SPLIT_WARPS 12
 #endif
@@ -88,7 +88,7 @@ struct LongTiles {
                        tile_bytes = TA_SPLIT_TILE_BYTES;
 };
 struct ShortTiles {
-  static constexpr int warps = 8, stages = 4, elems = 16, tile_bytes = 16384;
+  static constexpr int warps = 8, stages = 4, elems = 8, tile_bytes = 16384;
 };
 
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100 (227 KB)
@@ -111,7 +111,8 @@ struct SplitCfg {
   static constexpr int NSTAGE = V::stages;
   static constexpr int MERGE_BATCH = 128;      // partials whose weights are staged at once
   // Shared memory besides the ring: per-warp statistics, merge weights, barriers and flags.
-  static constexpr int FIXED_SMEM = NCW * G * D * 4 + 2 * NCW * G * 4 + MERGE_BATCH * G * 4 + 1024;
+  static constexpr int FIXED_SMEM =
+      NCW * G * D * 4 + 2 * NCW * G * 4 + MERGE_BATCH * G * 4 + NSTAGE * G * D * ELEM + 1024;
   static constexpr int MAX_TILE_BYTES = (kSmemLimit - FIXED_SMEM) / (2 * NSTAGE);
   static constexpr int TILE_TARGET = V::tile_bytes < MAX_TILE_BYTES ? V::tile_bytes : MAX_TILE_BYTES;
   static constexpr int STEPS_FIT = TILE_TARGET / (ROW * NCW * TPW);
@@ -136,6 +137,7 @@ template <class C>
 struct SplitSmem {
   alignas(128) uint8_t k[C::NSTAGE][C::TILE_BYTES];
   alignas(128) uint8_t v[C::NSTAGE][C::TILE_BYTES];
+  alignas(16) uint8_t q[C::NSTAGE][C::G * C::D * C::ELEM];  // q of a unit, copied with its first tile
   float wo[C::NCW][C::G][C::D];  // per-warp statistics of the current unit
   float wm[C::NCW][C::G];
   float wl[C::NCW][C::G];
@@ -323,10 +325,11 @@ __device__ __forceinline__ float tree_sum(const float (&a)[M]) {
   }
 }
 
-// out = O / L, lse = ln(2) (M + log2 L); an empty unit gives 0 and -inf; a unit
-// whose inputs may be incomplete (error word set) gives NaN.
+// out = O / L, lse = ln(2) (M + log2 L); an empty unit gives 0 and -inf; a unit whose
+// inputs may be incomplete (this CTA gave up waiting: `poisoned`) gives NaN.  NaN partials
+// of another CTA propagate through the merge weights (2^(NaN - M) is NaN).
 __device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq, int d, int D, float M, float L,
-                                            float O, bool write_lse) {
+                                            float O, bool write_lse, bool poisoned) {
   float ov, lv;
   if (L > 0.f) {
     ov = O / L;
@@ -335,7 +338,7 @@ __device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq,
     ov = 0.f;
     lv = -INFINITY;
   }
-  if (*reinterpret_cast<volatile int*>(p.err) != 0) {
+  if (poisoned || L != L) {
     ov = __int_as_float(0x7fc00000);
     lv = ov;
   }
@@ -401,8 +404,15 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
         const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - t0));
         if (!(cta == 0 && i == p.debug_skip_tile)) {
           const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
+          constexpr uint32_t q_bytes = G * D * C::ELEM;
+          const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
           uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
-          mbar_arrive_expect_tx(&sm.full[s], TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes);
+          mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
+          if (with_q) {
+            const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
+                                  (static_cast<int64_t>(w.b) * p.n_q_heads + w.h * G) * D * C::ELEM;
+            bulk_load(sm.q[s], qsrc, q_bytes, &sm.full[s], pol);
+          }
           if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
           if (bytes != 0) {
             const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
@@ -443,14 +453,15 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
     float2 o2[G][E2];  // unnormalised output of this lane's tokens
     float m = -INFINITY, l = 0.f;  // statistics of head head_of_lane(li) over this lane's tokens
 
-    auto load_q = [&](int b, int h) {
+    // The unit's q (landed in stage s with the unit's first tile), read like a K row so the
+    // register order matches the K elements it multiplies.
+    auto load_q = [&](int s) {
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const int64_t base = (static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * D;
+        RowLoader<T>::template load<C::NCH>(sm.q[s] + g * C::ROW, li, rot, q2[g]);
 #pragma unroll
-        for (int j = 0; j < E2; ++j)
-          q2[g][j] = make_float2(RowLoader<T>::scalar(p.q, base + dcol(2 * j)) * p.scale_log2,
-                                 RowLoader<T>::scalar(p.q, base + dcol(2 * j + 1)) * p.scale_log2);
+        for (int j = 0; j < E2; ++j) q2[g][j] = __fmul2_rn(q2[g][j], sc2);
       }
     };
     auto reset = [&]() {
@@ -502,6 +513,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
       named_barrier(1, C::NCT);
 
       // 2) merge the warps; write the final result or this CTA's partial
+      const bool poisoned = *abort_flag != 0;
       const int unit = b * p.n_kv_heads + h;
       const int64_t U0 = p.tile_off[b] + static_cast<int64_t>(h) * p.n_tiles[b];
       const int i_first = cta_of_tile(U0, NT, p.grid);
@@ -526,12 +538,13 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
           }
           const float O = tree_sum<C::NCW>(ao), L = tree_sum<C::NCW>(al);
           if (n_parts == 1) {
-            write_final(p, b, h * G + g, d, D, Mx, L, O, d == 0);
+            write_final(p, b, h * G + g, d, D, Mx, L, O, d == 0, poisoned);
           } else {
-            slot[2 * G + g * D + d] = O;
+            const float nan = __int_as_float(0x7fc00000);
+            slot[2 * G + g * D + d] = poisoned ? nan : O;
             if (d == 0) {
-              slot[g] = Mx;
-              slot[G + g] = L;
+              slot[g] = poisoned ? nan : Mx;
+              slot[G + g] = poisoned ? nan : L;
             }
           }
         }
@@ -568,10 +581,25 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
               const int col = tid + k * C::NCT;
               if (col < G * D) {
                 const int g = col / D, d = col % D;
-                for (int c = 0; c < nb; ++c) {
-                  const float* sp = base + static_cast<int64_t>(c0 + c) * C::SLOT;
-                  acc[k].push(sm.mw[c][g] * ld_cg(sp + 2 * G + g * D + d));
-                  if (d == 0) accl[k].push(sm.mw[c][g] * ld_cg(sp + G + g));
+                // Leaves in batches of 16: the batch's loads are in flight together, then
+                // enter the pairwise sum in order.
+                constexpr int LB = 16;
+                for (int cb = 0; cb < nb; cb += LB) {
+                  float ov[LB], lv[LB];
+#pragma unroll
+                  for (int u = 0; u < LB; ++u) {
+                    const bool in = cb + u < nb;
+                    const float* sp = base + static_cast<int64_t>(c0 + cb + u) * C::SLOT;
+                    ov[u] = in ? ld_cg(sp + 2 * G + g * D + d) : 0.f;
+                    lv[u] = (in && d == 0) ? ld_cg(sp + G + g) : 0.f;
+                  }
+#pragma unroll
+                  for (int u = 0; u < LB; ++u) {
+                    if (cb + u < nb) {
+                      acc[k].push(sm.mw[cb + u][g] * ov[u]);
+                      if (d == 0) accl[k].push(sm.mw[cb + u][g] * lv[u]);
+                    }
+                  }
                 }
               }
             }
@@ -588,7 +616,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
             const int col = tid + k * C::NCT;
             if (col < G * D) {
               const int g = col / D, d = col % D;
-              write_final(p, b, h * G + g, d, D, sm.mM[g], sm.mL[g], acc[k].result(), d == 0);
+              write_final(p, b, h * G + g, d, D, sm.mM[g], sm.mL[g], acc[k].result(), d == 0, poisoned);
             }
           }
           if (tid == 0) p.tickets[unit] = 0;
@@ -600,16 +628,16 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
     TileWalk w;
     w.init(p, t_lo);
     int cur_b = w.b, cur_h = w.h;
-    load_q(cur_b, cur_h);
     reset();
+    bool new_unit = true;
 
     for (int i = 0; i < n_my; ++i) {
       if (w.b != cur_b || w.h != cur_h) {
         finalize(cur_b, cur_h);
         cur_b = w.b;
         cur_h = w.h;
-        load_q(cur_b, cur_h);
         reset();
+        new_unit = true;
       }
       const int s = i % C::NSTAGE;
       bool ok = (*abort_flag == 0);
@@ -618,6 +646,10 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
       if (!ok && lane == 0) {
         if (!*abort_flag) atomicCAS(p.err, 0, kErrConsumerWait);
         *abort_flag = 1;
+      }
+      if (ok && new_unit) {
+        load_q(s);
+        new_unit = false;
       }
       if (ok) {
         const int64_t len = p.seq_len[w.b];
