@@ -13,15 +13,17 @@
 // Each CTA writes per row the statistics (m in log2 units, l, unnormalised o) of its
 // chunk; merge_prefix_suffix_kernel combines the chunks with the suffix part.
 //
-// One CTA owns up to 256 rows (two M tiles of 128) and a contiguous chunk of 64-key
+// One CTA owns up to 256 rows (two M tiles of 128) and a contiguous chunk of 128-key
 // tiles of the context; both M tiles consume every K/V tile it loads.
-// Roles (13 warps):  warp 0 lane 0 / warp 12 lane 0: TMA producers of the K and of the V
-// tiles (K stages free as soon as QK is done, V stages only after P V);  warp 1: TMEM
-// allocation and lane 0 issues tcgen05.mma;  warps 2-3: convert each V tile from bf16
-// to fp16 in place (P is kept in fp16 for the P V product: bf16 P is too coarse);
-// warps 4-7 and 8-11: softmax of M tile 0 and 1, thread t owns row t = TMEM lane t.
-// TMEM columns: S of tile w, buffer b at 128 w + 64 b (fp32, 128 x 64); O of tile w at
-// 256 + 128 w (128 x 128).
+// Roles (12 warps):  warp 0 lane 0: TMA producer (K and V streams, each refilling a stage
+// once its own product freed it);  warp 1: TMEM allocation, lane 0 issues tcgen05.mma;
+// warps 2-3: convert each V tile from bf16 to fp16 in place (P is fp16 for the P V
+// product: bf16 P is too coarse, and one MMA needs A and B of the same type);  warps 4-7
+// and 8-11: softmax of M tile 0 and 1, thread t owns row t = TMEM lane t.
+// TMEM columns: S of tile w at 128 w (fp32, 128 x 128); P (fp16, two per column)
+// overwrites its first 64 columns and is the A operand of P V; O of tile w at 256 + 128 w.
+// Per M tile the MMA thread alternates S(t) = Q K(t)^T and O += P(t) V(t); the tensor pipe
+// runs them in issue order, so S(t + 1) landing also means P(t) V(t) is complete.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -35,24 +37,24 @@ namespace ta {
 
 constexpr int kBifRows = 128;       // rows of one M tile (one TMEM lane each)
 constexpr int kBifMT = 2;           // M tiles per CTA: the CTA's 256 rows share every K/V tile
-constexpr int kBifKeys = 64;        // keys per tile (N of S, K of P V)
+constexpr int kBifKeys = 128;       // keys per tile (N of S, K of P V)
 constexpr int kBifD = 128;          // head_dim
-constexpr int kBifStages = 3;       // K ring and V ring depth
-constexpr int kBifThreads = 416;    // 13 warps
-constexpr int kBifTmemCols = 512;   // S: 2 tiles x 2 buffers x 64 columns; O: 2 tiles x 128 columns
+constexpr int kBifKStages = 3;      // K ring depth (K frees a stage after S = Q K^T)
+constexpr int kBifVStages = 2;      // V ring depth (V frees a stage after O += P V)
+constexpr int kBifThreads = 384;    // 12 warps
+constexpr int kBifTmemCols = 512;   // S: 2 tiles x 128 columns; O: 2 tiles x 128 columns
 constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
 
 constexpr int kErrBifWait = 4;
 constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
 
 struct BifSmem {
-  alignas(1024) uint8_t q[kBifMT][2][kBifRows * 128];      // bf16 Q tiles, two 64-column blocks each, SW128
-  alignas(1024) uint8_t k[kBifStages][2][kBifKeys * 128];  // bf16 K tiles, two 64-column blocks
-  alignas(1024) uint8_t v[kBifStages][2][kBifKeys * 128];  // V tiles (bf16 -> fp16 in place), MN-major
-  alignas(1024) uint8_t p[kBifMT][2][kBifRows * 128];      // fp16 P per M tile, double buffered, SW128
-  uint64_t k_full[kBifStages], v_full[kBifStages], v_conv[kBifStages];
-  uint64_t k_empty[kBifStages], v_empty[kBifStages];
-  uint64_t s_full[kBifMT][2], s_free[kBifMT][2], p_full[kBifMT][2], pv_done[kBifMT][2];
+  alignas(1024) uint8_t q[kBifMT][2][kBifRows * 128];        // bf16 Q tiles, two 64-column blocks each, SW128
+  alignas(1024) uint8_t k[kBifKStages][2][kBifKeys * 128];   // bf16 K tiles, two 64-column blocks
+  alignas(1024) uint8_t v[kBifVStages][2][kBifKeys * 128];   // V tiles (bf16 -> fp16 in place), MN-major
+  uint64_t k_full[kBifKStages], k_empty[kBifKStages];
+  uint64_t v_full[kBifVStages], v_conv[kBifVStages], v_empty[kBifVStages];
+  uint64_t s_full[kBifMT], p_full[kBifMT], o_done[kBifMT];
   uint64_t q_ready, mma_idle;
   uint32_t tmem_base;
   int abort;
@@ -105,6 +107,20 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] x B[smem desc]; A is K-major in TMEM (row = lane, two 16-bit
+// elements per 32-bit column).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z), "r"(z), "r"(z), "r"(z)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05.mma issued so far by this thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
@@ -141,6 +157,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 
@@ -207,22 +234,22 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 
   if (tid == 0) {
 #pragma unroll
-    for (int s = 0; s < kBifStages; ++s) {
+    for (int s = 0; s < kBifKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.v_conv[s], 64);
-      mbar_init(&sm.k_empty[s], 1);
-      mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.k_empty[s], n_mt);  // one commit per active M tile's S = Q K^T
     }
 #pragma unroll
-    for (int w = 0; w < kBifMT; ++w)
+    for (int s = 0; s < kBifVStages; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_conv[s], 64);
+      mbar_init(&sm.v_empty[s], n_mt);  // one commit per active M tile's O += P V
+    }
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&sm.s_full[w][b], 1);
-        mbar_init(&sm.s_free[w][b], kBifRows);
-        mbar_init(&sm.p_full[w][b], kBifRows);
-        mbar_init(&sm.pv_done[w][b], 1);
-      }
+    for (int w = 0; w < kBifMT; ++w) {
+      mbar_init(&sm.s_full[w], 1);
+      mbar_init(&sm.p_full[w], kBifRows);
+      mbar_init(&sm.o_done[w], 1);
+    }
     mbar_init(&sm.q_ready, kBifMT * kBifRows);
     mbar_init(&sm.mma_idle, 1);
     sm.abort = 0;
@@ -240,32 +267,50 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 0 || warp == 12) {
-    // ------------------------------- TMA producers ------------------------------
-    // warp 0 streams K, warp 12 streams V; each refills a stage once its own product freed it.
+  if (warp == 0) {
+    // ------------------------------- TMA producer -------------------------------
+    // Two streams in tile order; a K stage refills once both M tiles' S = Q K^T read it, a
+    // V stage once both M tiles' P V read it.  Whichever stream can proceed is issued.
     if (lane == 0) {
-      const bool is_k = warp == 0;
-      uint64_t* full = is_k ? sm.k_full : sm.v_full;
-      uint64_t* empty = is_k ? sm.k_empty : sm.v_empty;
-      const CUtensorMap* map = is_k ? &kmap : &vmap;
       uint64_t pol;
       asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-      int fills = 0;
-      for (int i = 0; i < n_t; ++i) {
-        const int s = i % kBifStages;
-        if (i >= kBifStages && !bif_wait(&empty[s], ((i / kBifStages) - 1) & 1, p, abort)) break;
-        if (*abort) break;
-        const int y = static_cast<int>(h * p.prefix_len + (j0 + i) * kBifKeys);
-        uint8_t* dst = is_k ? sm.k[s][0] : sm.v[s][0];
-        mbar_arrive_expect_tx(&full[s], 2 * kBifKeys * 128);
-        tma_load_2d(dst, map, 0, y, &full[s], pol);
-        tma_load_2d(dst + kBifKeys * 128, map, 64, y, &full[s], pol);
-        ++fills;
+      auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int t) {
+        const int y = static_cast<int>(h * p.prefix_len + (j0 + t) * kBifKeys);
+        mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
+        tma_load_2d(dst, map, 0, y, full, pol);
+        tma_load_2d(dst + kBifKeys * 128, map, 64, y, full, pol);
+      };
+      int tk = 0, tv = 0;
+      uint64_t t_idle = global_timer_ns();
+      while ((tk < n_t || tv < n_t) && !*abort) {
+        bool progress = false;
+        if (tk < n_t && (tk < kBifKStages ||
+                         mbar_test_wait(&sm.k_empty[tk % kBifKStages], ((tk / kBifKStages) - 1) & 1))) {
+          issue(&kmap, sm.k[tk % kBifKStages][0], &sm.k_full[tk % kBifKStages], tk);
+          ++tk;
+          progress = true;
+        }
+        if (tv < n_t && (tv < kBifVStages ||
+                         mbar_test_wait(&sm.v_empty[tv % kBifVStages], ((tv / kBifVStages) - 1) & 1))) {
+          issue(&vmap, sm.v[tv % kBifVStages][0], &sm.v_full[tv % kBifVStages], tv);
+          ++tv;
+          progress = true;
+        }
+        if (progress) {
+          t_idle = global_timer_ns();
+        } else if (static_cast<int64_t>(global_timer_ns() - t_idle) > p.wait_limit_ns) {
+          atomicCAS(p.err, 0, kErrBifWait);
+          *abort = 1;
+        }
       }
       // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
-      for (int s = 0; s < kBifStages && s < fills; ++s) {
-        const int last = (fills - 1 - s) / kBifStages;
-        if (!wait_phase(&full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+      for (int s = 0; s < kBifKStages && s < tk; ++s) {
+        const int last = (tk - 1 - s) / kBifKStages;
+        if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+      }
+      for (int s = 0; s < kBifVStages && s < tv; ++s) {
+        const int last = (tv - 1 - s) / kBifVStages;
+        if (!wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
       }
     }
     __syncwarp();
@@ -276,75 +321,52 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       constexpr uint32_t idesc_pv = f16_idesc(kBifRows, kBifD, false, false, true);
       bool ok = bif_wait(&sm.q_ready, 0, p, abort);
       tc_fence_after();
-      // S = Q K^T of tile t into S buffer t & 1 of every active M tile.
-      auto issue_qk = [&](int t) -> bool {
-        const int s = t % kBifStages, b = t & 1;
-        if (!bif_wait(&sm.k_full[s], (t / kBifStages) & 1, p, abort)) return false;
-        const uint32_t k_base = smem_addr(sm.k[s]);
-        for (int w = 0; w < n_mt; ++w) {
-          // Buffer b last held tile t - 2; its softmax has loaded it once s_free fires.
-          if (t >= 2 && !bif_wait(&sm.s_free[w][b], ((t - 2) >> 1) & 1, p, abort)) return false;
-          tc_fence_after();
-          const uint32_t q_base = smem_addr(sm.q[w]);
-#pragma unroll
-          for (int kk = 0; kk < kBifD / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
-            const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
-            const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
-            tc_mma_f16(tmem + w * 128 + b * kBifKeys, a, bd, idesc_qk, kk > 0);
-          }
-          tc_commit(&sm.s_full[w][b]);
-        }
-        tc_commit(&sm.k_empty[s]);
-        return true;
-      };
-      // O += P V of tile t for every active M tile.
-      auto issue_pv = [&](int t) -> bool {
-        const int s = t % kBifStages, b = t & 1;
-        if (!bif_wait(&sm.v_conv[s], (t / kBifStages) & 1, p, abort)) return false;
-        const uint32_t v_base = smem_addr(sm.v[s]);
-        for (int w = 0; w < n_mt; ++w) {
-          if (!bif_wait(&sm.p_full[w][b], (t >> 1) & 1, p, abort)) return false;
-          tc_fence_after();
-          const uint32_t p_base = smem_addr(sm.p[w][b]);
-#pragma unroll
-          for (int kk = 0; kk < kBifKeys / 16; ++kk) {
-            const uint64_t a = sw128_desc(p_base + kk * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
-            tc_mma_f16(tmem + 256 + w * 128, a, bd, idesc_pv, t > 0 || kk > 0);
-          }
-          tc_commit(&sm.pv_done[w][b]);
-        }
-        tc_commit(&sm.v_empty[s]);
-        return true;
-      };
-      // Two streams, QK(tq) and PV(tp), each in tile order; whichever has its inputs ready
-      // is issued, so neither waits for the other (the tensor pipe runs them in issue order).
-      // QK(t) needs K(t) and the softmax of t - 2 to have loaded its S buffer; PV(t) needs
-      // V(t) converted and P(t) written.
-      auto qk_ready = [&](int t) {
-        if (!mbar_test_wait(&sm.k_full[t % kBifStages], (t / kBifStages) & 1)) return false;
-        for (int w = 0; t >= 2 && w < n_mt; ++w)
-          if (!mbar_test_wait(&sm.s_free[w][t & 1], ((t - 2) >> 1) & 1)) return false;
-        return true;
-      };
-      auto pv_ready = [&](int t) {
-        if (!mbar_test_wait(&sm.v_conv[t % kBifStages], (t / kBifStages) & 1)) return false;
+      // Per M tile w the stream is S(0), PV(0), S(1), PV(1), ...: S(t + 1) overwrites the
+      // TMEM columns where P(t) was read, so it follows P(t) V(t) in issue order.
+      int tq[kBifMT] = {0, 0}, tp[kBifMT] = {0, 0};
+      auto all_done = [&]() {
         for (int w = 0; w < n_mt; ++w)
-          if (!mbar_test_wait(&sm.p_full[w][t & 1], (t >> 1) & 1)) return false;
+          if (tp[w] < n_t) return false;
         return true;
       };
-      int tq = 0, tp = 0;
       uint64_t t_idle = global_timer_ns();
-      while (ok && tp < n_t) {
+      while (ok && !all_done()) {
         bool progress = false;
-        if (tq < n_t && qk_ready(tq)) {
-          ok = issue_qk(tq++);
-          progress = true;
-        }
-        if (ok && tp < tq && pv_ready(tp)) {
-          ok = issue_pv(tp++);
-          progress = true;
+        for (int w = 0; w < n_mt; ++w) {
+          if (tq[w] == tp[w] && tq[w] < n_t) {
+            const int t = tq[w], s = t % kBifKStages;
+            if (mbar_test_wait(&sm.k_full[s], (t / kBifKStages) & 1)) {
+              tc_fence_after();
+              const uint32_t q_base = smem_addr(sm.q[w]);
+              const uint32_t k_base = smem_addr(sm.k[s]);
+#pragma unroll
+              for (int kk = 0; kk < kBifD / 16; ++kk) {
+                const uint32_t off = (kk & 3) * 32;  // 16-element K step inside a 128-byte row
+                const uint64_t a = sw128_desc(q_base + (kk >> 2) * (kBifRows * 128) + off, 16, 1024);
+                const uint64_t bd = sw128_desc(k_base + (kk >> 2) * (kBifKeys * 128) + off, 16, 1024);
+                tc_mma_f16(tmem + w * 128, a, bd, idesc_qk, kk > 0);
+              }
+              tc_commit(&sm.s_full[w]);
+              tc_commit(&sm.k_empty[s]);
+              ++tq[w];
+              progress = true;
+            }
+          } else if (tp[w] < tq[w]) {
+            const int t = tp[w], s = t % kBifVStages;
+            if (mbar_test_wait(&sm.v_conv[s], (t / kBifVStages) & 1) && mbar_test_wait(&sm.p_full[w], t & 1)) {
+              tc_fence_after();
+              const uint32_t v_base = smem_addr(sm.v[s]);
+#pragma unroll
+              for (int kk = 0; kk < kBifKeys / 16; ++kk) {
+                const uint64_t bd = sw128_desc(v_base + kk * 16 * 128, kBifKeys * 128, 1024);
+                tc_mma_f16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, bd, idesc_pv, t > 0 || kk > 0);
+              }
+              tc_commit(&sm.v_empty[s]);
+              if (t == n_t - 1) tc_commit(&sm.o_done[w]);
+              ++tp[w];
+              progress = true;
+            }
+          }
         }
         if (progress) {
           t_idle = global_timer_ns();
@@ -365,8 +387,8 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     // ------------------------------- V converters -------------------------------
     const int ct = tid - 64;
     for (int i = 0; i < n_t; ++i) {
-      const int s = i % kBifStages;
-      if (!bif_wait(&sm.v_full[s], (i / kBifStages) & 1, p, abort)) break;
+      const int s = i % kBifVStages;
+      if (!bif_wait(&sm.v_full[s], (i / kBifVStages) & 1, p, abort)) break;
       uint4* v4 = reinterpret_cast<uint4*>(sm.v[s]);
 #pragma unroll 4
       for (int c = ct; c < 2 * kBifKeys * 128 / 16; c += 64) {
@@ -409,31 +431,25 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = w < n_mt;
     for (int i = 0; ok && i < n_t; ++i) {
-      const int b = i & 1;
-      ok = bif_wait(&sm.s_full[w][b], (i >> 1) & 1, p, abort);
+      // S(i) landed; with it, P(i - 1) V(i - 1) is complete (same issuing thread, in order).
+      ok = bif_wait(&sm.s_full[w], i & 1, p, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       float x[kBifKeys];
-      {
+#pragma unroll
+      for (int q4 = 0; q4 < kBifKeys / 32; ++q4) {
         float t[32];
-        tmem_ld32(s_col + b * kBifKeys, t);
+        tmem_ld32(s_col + q4 * 32, t);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = t[c];
-        tmem_ld32(s_col + b * kBifKeys + 32, t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 + c] = t[c];
-        tmem_wait_ld();
+        for (int c = 0; c < 32; ++c) x[q4 * 32 + c] = t[c];
       }
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[w][b]);
+      tmem_wait_ld();
       const int64_t nvalid = p.prefix_len - (j0 + i) * kBifKeys;
-      uint32_t ph[kBifKeys / 2];
-      float mn, rs;
-      bool need;
-      if (nvalid >= kBifKeys) {
-        // Full tile: scaled max from the raw extreme, then p = 2^(x s - m) with one FFMA each.
-        // Extreme of the raw scores in 8 independent chains, then a tree.
+      const bool full = nvalid >= kBifKeys;
+      float tmax;
+      if (full) {
+        // Scaled max from the raw extreme (8 independent chains, then a tree).
         float xe[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) xe[k] = x[k];
@@ -452,58 +468,48 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 #pragma unroll
             for (int j = 0; j < k; ++j) xe[j] = fminf(xe[j], xe[j + k]);
         }
-        const float tmax = xe[0] * sc;
-        need = tmax > m + kBifRescale;
-        mn = need ? tmax : m;
-        const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < kBifKeys; c += 2) {
-          const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), s2, nm);
-          const float2 pp = make_float2(ex2(y.x), ex2(y.y));
-          acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], pp);
-          const __half2 hv = __floats2half2_rn(pp.x, pp.y);
-          ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-        const float2 a = __fadd2_rn(a01, a23);
-        rs = a.x + a.y;
+        tmax = xe[0] * sc;
       } else {
         // Last, partial tile of the context: keys past its end get p = 0.
-        float tmax = -INFINITY;
+        tmax = -INFINITY;
 #pragma unroll
         for (int c = 0; c < kBifKeys; ++c) {
           x[c] = (c < nvalid) ? x[c] * sc : -INFINITY;
           tmax = fmaxf(tmax, x[c]);
         }
-        need = tmax > m + kBifRescale;
-        mn = need ? tmax : m;
-        rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < kBifKeys; c += 2) {
-          const float p0 = (x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn);
-          const float p1 = (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn);
-          rs += p0 + p1;
-          const __half2 hv = __floats2half2_rn(p0, p1);
-          ph[c / 2] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
       }
-      // P buffer b was last read by the P V product of tile i - 2.
-      if (i >= 2) ok = bif_wait(&sm.pv_done[w][b], ((i - 2) >> 1) & 1, p, abort);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
+      const bool need = tmax > m + kBifRescale;
+      const float mn = need ? tmax : m;
+      // p = 2^(x s - m) (one packed FFMA per pair on full tiles), summed in fp32 and written
+      // as fp16 pairs over the first 64 columns of S, half a tile at a time.
+      const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(sm.p[w][b] + sw128_offset(r, c)) =
-            make_uint4(ph[4 * c], ph[4 * c + 1], ph[4 * c + 2], ph[4 * c + 3]);
-      fence_proxy_async_smem();
+      for (int half = 0; half < 2; ++half) {
+        uint32_t t[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = half * 64 + 2 * c2;
+          float2 pp;
+          if (full) {
+            const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), s2, nm);
+            pp = make_float2(ex2(y.x), ex2(y.y));
+          } else {
+            pp = make_float2((x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn),
+                             (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn));
+          }
+          acc[c2 & 3] = __fadd2_rn(acc[c2 & 3], pp);
+          const __half2 hv = __floats2half2_rn(pp.x, pp.y);
+          t[c2] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        tmem_st32u(s_col + half * 32, t);
+      }
+      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 a4 = __fadd2_rn(a01, a23);
+      const float rs = a4.x + a4.y;
       const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
-      // O holds tiles 0..i-1: rescale it (after the P V product of tile i-1) when m grew.
+      // O holds tiles 0..i-1 and P(i - 1) V(i - 1) is complete: rescale it when m grew.
       if (__any_sync(0xffffffffu, need && i >= 1)) {
-        ok = bif_wait(&sm.pv_done[w][(i - 1) & 1], ((i - 1) >> 1) & 1, p, abort);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
 #pragma unroll
         for (int q4 = 0; q4 < kBifD / 32; ++q4) {
           float o[32];
@@ -513,19 +519,19 @@ __global__ void __launch_bounds__(kBifThreads, 1)
           for (int c = 0; c < 32; ++c) o[c] *= alpha;
           tmem_st32(o_col + q4 * 32, o);
         }
-        tmem_wait_st();
       }
+      tmem_wait_st();
       l = l * alpha + rs;
       m = mn;
       tc_fence_before();
-      mbar_arrive(&sm.p_full[w][b]);
+      mbar_arrive(&sm.p_full[w]);
     }
     // The chunk's statistics of this row.
     if (w < n_mt) {
       float* dst =
           p.part + ((static_cast<int64_t>(chunk) * p.n_kv_heads + h) * p.rows_per_head + row) * kBifPartRow;
       if (n_t > 0 && ok) {
-        ok = bif_wait(&sm.pv_done[w][(n_t - 1) & 1], ((n_t - 1) >> 1) & 1, p, abort);
+        ok = bif_wait(&sm.o_done[w], 0, p, abort);
         ok = __all_sync(0xffffffffu, ok);
       }
       if (n_t > 0 && ok) {

@@ -56,6 +56,7 @@ struct SplitParams {
   int32_t n_q_heads;
   float scale_log2;       // scale * log2(e): scores come out in base-2 units
   int32_t debug_skip_tile;
+  int32_t unit_aligned;   // 1: CTA ranges start at unit boundaries, so no unit is shared by CTAs
   int64_t kv_off[kMaxSeqPerLaunch];
   int64_t seq_len[kMaxSeqPerLaunch];
   int64_t tile_off[kMaxSeqPerLaunch + 1];  // first tile of sequence b on the line
@@ -296,6 +297,17 @@ __device__ __forceinline__ int cta_of_tile(int64_t t, int64_t NT, int P) {
   return static_cast<int>(((t + 1) * P - 1) / NT);
 }
 
+// First tile of CTA i: i*NT/P, rounded up to the next (sequence, KV head) unit start when the
+// plan keeps units whole.
+__device__ __forceinline__ int64_t cta_first_tile(const SplitParams& p, int i) {
+  const int64_t NT = p.n_tiles_total;
+  const int64_t t = static_cast<int64_t>(i) * NT / p.grid;
+  if (!p.unit_aligned || t >= NT) return t;
+  TileWalk w;
+  w.init(p, t);
+  return w.j == 0 ? t : t - w.j + p.n_tiles[w.b];
+}
+
 // Sum of leaves in a fixed pairwise tree: leaf n is combined with the pending
 // subtrees as a binary counter carries, so the shape depends only on the leaf count.
 struct PairwiseSum {
@@ -364,8 +376,8 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
   const int lane = tid & 31;
   const int cta = blockIdx.x;
   const int64_t NT = p.n_tiles_total;
-  const int64_t t_lo = static_cast<int64_t>(cta) * NT / p.grid;
-  const int64_t t_hi = static_cast<int64_t>(cta + 1) * NT / p.grid;
+  const int64_t t_lo = cta_first_tile(p, cta);
+  const int64_t t_hi = cta_first_tile(p, cta + 1);
   const int n_my = static_cast<int>(t_hi - t_lo);
 
   if (tid == 0) {
@@ -518,7 +530,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
       const int64_t U0 = p.tile_off[b] + static_cast<int64_t>(h) * p.n_tiles[b];
       const int i_first = cta_of_tile(U0, NT, p.grid);
       const int i_last = cta_of_tile(U0 + p.n_tiles[b] - 1, NT, p.grid);
-      const int n_parts = i_last - i_first + 1;
+      const int n_parts = p.unit_aligned ? 1 : i_last - i_first + 1;
       float* slot = p.part + static_cast<int64_t>(cta + unit) * C::SLOT;
 #pragma unroll
       for (int k = 0; k < C::NCOL; ++k) {

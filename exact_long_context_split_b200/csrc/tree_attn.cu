@@ -126,6 +126,7 @@ ta_status resident_ctas(const KernelInfo& ki, int* device_out, int* slots_out) {
 struct Group {
   int b0 = 0, nb = 0;
   int P = 0;
+  bool unit_aligned = false;
   int64_t NT = 0;
   size_t tickets_off = 0, part_off = 0;  // byte offsets inside the workspace body
   int64_t kv_off[kMaxSeqPerLaunch];
@@ -166,6 +167,11 @@ ta_status build_plan(const int64_t* seqlens, const int64_t* kv_offsets, int batc
     P = std::max<int64_t>(1, std::min<int64_t>(P, NT));
     g.P = static_cast<int>(P);
     const int64_t units = static_cast<int64_t>(g.nb) * Hkv;
+    // Many short units: keep each unit in one CTA (no partials, tickets or merge tails) when
+    // every unit is at most half a CTA's share of tiles, so the ranges stay balanced.
+    int32_t max_unit_tiles = 0;
+    for (int i = 0; i < g.nb; ++i) max_unit_tiles = std::max(max_unit_tiles, g.n_tiles[i]);
+    g.unit_aligned = units >= P && 2 * static_cast<int64_t>(max_unit_tiles) * P <= NT;
     g.tickets_off = body;
     body = align_up(body + sizeof(int) * units, kAlign);
     g.part_off = body;
@@ -247,6 +253,7 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
     p.n_q_heads = Hq;
     p.scale_log2 = static_cast<float>(s2);
     p.debug_skip_tile = opts ? opts->debug_skip_tile : -1;
+    p.unit_aligned = g.unit_aligned ? 1 : 0;
     for (int i = 0; i < g.nb; ++i) {
       p.kv_off[i] = g.kv_off[i];
       p.seq_len[i] = g.len[i];
