@@ -1,0 +1,29 @@
+// The bifurcated tensor-core kernels and their launchers.
+#include "bifurcated_tc.cuh"
+
+namespace ta {
+
+size_t bif_prefix_smem_bytes() { return sizeof(BifSmem) + 1024; }
+
+cudaError_t bif_prefix_set_smem_limit() {
+  return cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bif_prefix_smem_bytes()));
+}
+
+cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensorMap& vmap, const BifParams& p,
+                              cudaStream_t st) {
+  bif_prefix_kernel<<<grid, kBifThreads, bif_prefix_smem_bytes(), st>>>(kmap, vmap, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,
+                                       const float* out_s, const float* lse_s, float* out, float* lse,
+                                       int n_samples, int n_q_heads, const int* err, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(n_samples) * n_q_heads * (kBifD / 4);  // one thread per 4 columns
+  if (n == 0) return cudaSuccess;
+  merge_prefix_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      part, n_chunks, n_kv_heads, rows_per_head, out_s, lse_s, out, lse, n_samples, n_q_heads, err);
+  return cudaGetLastError();
+}
+
+}  // namespace ta

@@ -31,22 +31,18 @@
 
 #include <cstdint>
 
+#include "bifurcated_tc.h"
 #include "ptx.cuh"
 
 namespace ta {
 
-constexpr int kBifRows = 128;       // rows of one M tile (one TMEM lane each)
-constexpr int kBifMT = 2;           // M tiles per CTA: the CTA's 256 rows share every K/V tile
-constexpr int kBifKeys = 128;       // keys per tile (N of S, K of P V)
-constexpr int kBifD = 128;          // head_dim
 constexpr int kBifKStages = 3;      // K ring depth (K frees a stage after S = Q K^T)
 constexpr int kBifVStages = 2;      // V ring depth (V frees a stage after O += P V)
-constexpr int kBifThreads = 384;    // 12 warps
 constexpr int kBifTmemCols = 512;   // S: 2 tiles x 128 columns; O: 2 tiles x 128 columns
 constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
+constexpr bool kBifPingPong = true;  // the two softmax warpgroups take turns on the exponentials
+constexpr int kBifPolyEvery = 0;     // every k-th pair of exponentials on the FMA pipe (0: none)
 
-constexpr int kErrBifWait = 4;
-constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
 
 struct BifSmem {
   alignas(1024) uint8_t q[kBifMT][2][kBifRows * 128];        // bf16 Q tiles, two 64-column blocks each, SW128
@@ -55,24 +51,12 @@ struct BifSmem {
   uint64_t k_full[kBifKStages], k_empty[kBifKStages];
   uint64_t v_full[kBifVStages], v_conv[kBifVStages], v_empty[kBifVStages];
   uint64_t s_full[kBifMT], p_full[kBifMT], o_done[kBifMT];
+  uint64_t turn[kBifMT];  // turn[w] completes a phase when the other M tile's exponentials are done
   uint64_t q_ready, mma_idle;
   uint32_t tmem_base;
   int abort;
 };
 
-struct BifParams {
-  const void* q;          // [N][Hq][D] bf16
-  float* part;            // [chunks][Hkv * rows_per_head][kBifPartRow]: m (log2), l, -, -, o[D]
-  int* err;
-  int n_samples;
-  int n_q_heads;
-  int n_kv_heads;
-  int rows_per_head;      // N * G
-  int n_chunks;
-  int64_t prefix_len;
-  float scale_log2;
-  int64_t wait_limit_ns;
-};
 
 // ---------------------------------------------------------------------------------------------
 // PTX wrappers (tcgen05, TMA tensor loads, proxy fences)
@@ -200,6 +184,183 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
+// 2^y for a pair, on the FMA pipe: y = j + f with j = rint(y) (the 1.5 * 2^23 rounding
+// trick) and f in [-1/2, 1/2]; 2^f from a degree-4 polynomial fitted here to the relative
+// error of 2^f on that interval (weighted least squares, max relative error 2.7e-6 with
+// float32 Horner evaluation); j is added to the exponent field.  y below -126 is clamped
+// (its power of two is below every value a softmax weight can contribute here).
+__device__ __forceinline__ float2 exp2_poly2(float2 y) {
+  y.x = fmaxf(y.x, -126.f);
+  y.y = fmaxf(y.y, -126.f);
+  const float2 t = __fadd2_rn(y, make_float2(12582912.f, 12582912.f));
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), y);
+  float2 q = __ffma2_rn(make_float2(0.009570068679749966f, 0.009570068679749966f), f,
+                        make_float2(0.055917806923389435f, 0.055917806923389435f));
+  q = __ffma2_rn(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  q = __ffma2_rn(q, f, make_float2(0.6931218504905701f, 0.6931218504905701f));
+  q = __ffma2_rn(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// 3-input max / min (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// tcgen05.wait::ld that also hands the loaded registers through, so no use of them can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(float (&v)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]), "+f"(v[8]),
+        "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]),
+        "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]), "+f"(v[24]),
+        "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+      :
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Scaled max of a full tile's 128 scores (the raw extreme times the scale: for a negative
+// scale the raw minimum), two 32-column loads at a time, four independent chains.
+__device__ __forceinline__ float bif_tile_max(uint32_t s_col, float sc) {
+  float a[32], b[32];
+  float e[4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    tmem_ld32(s_col + 64 * h, a);
+    tmem_ld32(s_col + 64 * h + 32, b);
+    tmem_wait_ld_regs(a);
+    tmem_wait_ld_regs(b);
+    if (h == 0) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e[k] = a[k];
+    }
+    if (sc >= 0.f) {
+#pragma unroll
+      for (int c = (h == 0 ? 4 : 0); c < 32; c += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) e[k] = fmax3(e[k], a[c + k], c + k + 4 < 32 ? a[c + k + 4] : a[c + k]);
+      }
+#pragma unroll
+      for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) e[k] = fmax3(e[k], b[c + k], b[c + k + 4]);
+      }
+    } else {
+#pragma unroll
+      for (int c = (h == 0 ? 4 : 0); c < 32; c += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) e[k] = fmin3(e[k], a[c + k], c + k + 4 < 32 ? a[c + k + 4] : a[c + k]);
+      }
+#pragma unroll
+      for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) e[k] = fmin3(e[k], b[c + k], b[c + k + 4]);
+      }
+    }
+  }
+  const float x = sc >= 0.f ? fmax3(e[0], e[1], fmaxf(e[2], e[3])) : fmin3(e[0], e[1], fminf(e[2], e[3]));
+  return x * sc;
+}
+
+// The last, partial tile of the context: keys at or past `nvalid` do not exist.
+__device__ __forceinline__ float bif_tile_max_partial(uint32_t s_col, float sc, int nvalid) {
+  float tmax = -INFINITY;
+#pragma unroll 1
+  for (int q = 0; q < kBifKeys / 32; ++q) {
+    float a[32];
+    tmem_ld32(s_col + 32 * q, a);
+    tmem_wait_ld_regs(a);
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (32 * q + c < nvalid) tmax = fmaxf(tmax, a[c] * sc);
+  }
+  return tmax;
+}
+
+// 32 scores -> 16 fp16 pairs of p = 2^(x s - mn) at P columns [col, col + 16); adds p to acc.
+__device__ __forceinline__ void bif_exp_chunk(const float (&x)[32], uint32_t col, float2 s2, float2 nm,
+                                              float2 (&acc)[4]) {
+  uint32_t h[16];
+#pragma unroll
+  for (int c2 = 0; c2 < 16; ++c2) {
+    const float2 y = __ffma2_rn(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, nm);
+    float2 pp;
+    if (kBifPolyEvery > 0 && c2 % kBifPolyEvery == kBifPolyEvery - 1)
+      pp = exp2_poly2(y);
+    else
+      pp = make_float2(ex2(y.x), ex2(y.y));
+    acc[c2 & 3] = __fadd2_rn(acc[c2 & 3], pp);
+    const __half2 hv = __floats2half2_rn(pp.x, pp.y);
+    h[c2] = *reinterpret_cast<const uint32_t*>(&hv);
+  }
+  tmem_st16u(col, h);
+}
+
+// Pass 2 over a full tile: the next 32 scores load while the current ones are exponentiated.
+// P chunk q goes to columns [16 q, 16 q + 16), below every score column still to be read.
+__device__ __forceinline__ float bif_tile_exp(uint32_t s_col, float sc, float mn) {
+  const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float a[32], b[32];
+  tmem_ld32(s_col, a);
+  tmem_wait_ld_regs(a);
+  tmem_ld32(s_col + 32, b);
+  bif_exp_chunk(a, s_col, s2, nm, acc);
+  tmem_wait_ld_regs(b);
+  tmem_ld32(s_col + 64, a);
+  bif_exp_chunk(b, s_col + 16, s2, nm, acc);
+  tmem_wait_ld_regs(a);
+  tmem_ld32(s_col + 96, b);
+  bif_exp_chunk(a, s_col + 32, s2, nm, acc);
+  tmem_wait_ld_regs(b);
+  bif_exp_chunk(b, s_col + 48, s2, nm, acc);
+  const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 a4 = __fadd2_rn(a01, a23);
+  return a4.x + a4.y;
+}
+
+__device__ __forceinline__ float bif_tile_exp_partial(uint32_t s_col, float sc, float mn, int nvalid) {
+  float rs = 0.f;
+#pragma unroll 1
+  for (int q = 0; q < kBifKeys / 32; ++q) {
+    float a[32];
+    tmem_ld32(s_col + 32 * q, a);
+    tmem_wait_ld_regs(a);
+    uint32_t h[16];
+#pragma unroll
+    for (int c2 = 0; c2 < 16; ++c2) {
+      const int c = 32 * q + 2 * c2;
+      const float p0 = (c < nvalid) ? ex2(a[2 * c2] * sc - mn) : 0.f;
+      const float p1 = (c + 1 < nvalid) ? ex2(a[2 * c2 + 1] * sc - mn) : 0.f;
+      rs += p0 + p1;
+      const __half2 hv = __floats2half2_rn(p0, p1);
+      h[c2] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    tmem_st16u(s_col + 16 * q, h);
+  }
+  return rs;
+}
+
 // Bounded wait shared by every role: gives up after limit_ns or once the CTA aborted.
 __device__ __forceinline__ bool bif_wait(uint64_t* bar, uint32_t parity, const BifParams& p, volatile int* abort) {
   if (*abort) return false;
@@ -249,6 +410,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       mbar_init(&sm.s_full[w], 1);
       mbar_init(&sm.p_full[w], kBifRows);
       mbar_init(&sm.o_done[w], 1);
+      mbar_init(&sm.turn[w], kBifRows);
     }
     mbar_init(&sm.q_ready, kBifMT * kBifRows);
     mbar_init(&sm.mma_idle, 1);
@@ -436,77 +598,25 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      float x[kBifKeys];
-#pragma unroll
-      for (int q4 = 0; q4 < kBifKeys / 32; ++q4) {
-        float t[32];
-        tmem_ld32(s_col + q4 * 32, t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[q4 * 32 + c] = t[c];
-      }
-      tmem_wait_ld();
       const int64_t nvalid = p.prefix_len - (j0 + i) * kBifKeys;
       const bool full = nvalid >= kBifKeys;
-      float tmax;
-      if (full) {
-        // Scaled max from the raw extreme (8 independent chains, then a tree).
-        float xe[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) xe[k] = x[k];
-        if (sc >= 0.f) {
-#pragma unroll
-          for (int c = 8; c < kBifKeys; ++c) xe[c & 7] = fmaxf(xe[c & 7], x[c]);
-#pragma unroll
-          for (int k = 4; k >= 1; k >>= 1)
-#pragma unroll
-            for (int j = 0; j < k; ++j) xe[j] = fmaxf(xe[j], xe[j + k]);
-        } else {
-#pragma unroll
-          for (int c = 8; c < kBifKeys; ++c) xe[c & 7] = fminf(xe[c & 7], x[c]);
-#pragma unroll
-          for (int k = 4; k >= 1; k >>= 1)
-#pragma unroll
-            for (int j = 0; j < k; ++j) xe[j] = fminf(xe[j], xe[j + k]);
-        }
-        tmax = xe[0] * sc;
-      } else {
-        // Last, partial tile of the context: keys past its end get p = 0.
-        tmax = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kBifKeys; ++c) {
-          x[c] = (c < nvalid) ? x[c] * sc : -INFINITY;
-          tmax = fmaxf(tmax, x[c]);
-        }
-      }
+      // Pass 1: the tile's scaled row max, streamed from TMEM.
+      const float tmax = full ? bif_tile_max(s_col, sc) : bif_tile_max_partial(s_col, sc, static_cast<int>(nvalid));
       const bool need = tmax > m + kBifRescale;
       const float mn = need ? tmax : m;
-      // p = 2^(x s - m) (one packed FFMA per pair on full tiles), summed in fp32 and written
-      // as fp16 pairs over the first 64 columns of S, half a tile at a time.
-      const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t t[32];
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = half * 64 + 2 * c2;
-          float2 pp;
-          if (full) {
-            const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), s2, nm);
-            pp = make_float2(ex2(y.x), ex2(y.y));
-          } else {
-            pp = make_float2((x[c] == -INFINITY) ? 0.f : ex2(x[c] - mn),
-                             (x[c + 1] == -INFINITY) ? 0.f : ex2(x[c + 1] - mn));
-          }
-          acc[c2 & 3] = __fadd2_rn(acc[c2 & 3], pp);
-          const __half2 hv = __floats2half2_rn(pp.x, pp.y);
-          t[c2] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
-        tmem_st32u(s_col + half * 32, t);
+      // Ping-pong: M tile 1's exponentials of key tile i follow M tile 0's, and M tile 0's of
+      // tile i + 1 follow M tile 1's of tile i, so one warpgroup's exponentials overlap the
+      // other M tile's products on the tensor pipe.
+      const bool pingpong = kBifPingPong && n_mt == kBifMT;
+      if (pingpong && (w == 1 || i >= 1)) {
+        ok = bif_wait(&sm.turn[w], (w == 1 ? i : i - 1) & 1, p, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
       }
-      const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-      const float2 a4 = __fadd2_rn(a01, a23);
-      const float rs = a4.x + a4.y;
+      // Pass 2: p = 2^(x s - m), summed in fp32, written back as fp16 pairs over the first 64
+      // columns of S (P overwrites only columns whose scores were already read).
+      const float rs = full ? bif_tile_exp(s_col, sc, mn) : bif_tile_exp_partial(s_col, sc, mn, static_cast<int>(nvalid));
+      if (pingpong) mbar_arrive(&sm.turn[1 - w]);
       const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
       // O holds tiles 0..i-1 and P(i - 1) V(i - 1) is complete: rescale it when m grew.
       if (__any_sync(0xffffffffu, need && i >= 1)) {

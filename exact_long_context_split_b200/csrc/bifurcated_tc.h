@@ -1,0 +1,49 @@
+// Host-visible part of the bifurcated (shared-prefix) tensor-core pass: tile shapes, the
+// kernel parameters and the launchers; the kernels are in bifurcated_tc.cu.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace ta {
+
+constexpr int kBifRows = 128;       // rows of one M tile (one TMEM lane each)
+constexpr int kBifMT = 2;           // M tiles per CTA: the CTA's 256 rows share every K/V tile
+constexpr int kBifKeys = 128;       // keys per tile (N of S, K of P V)
+constexpr int kBifD = 128;          // head_dim
+constexpr int kBifThreads = 384;    // 12 warps
+constexpr int kErrBifWait = 4;
+constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
+
+struct BifParams {
+  const void* q;          // [N][Hq][D] bf16
+  float* part;            // [chunks][Hkv * rows_per_head][kBifPartRow]: m (log2), l, -, -, o[D]
+  int* err;
+  int n_samples;
+  int n_q_heads;
+  int n_kv_heads;
+  int rows_per_head;      // N * G
+  int n_chunks;
+  int64_t prefix_len;
+  float scale_log2;
+  int64_t wait_limit_ns;
+};
+
+// Dynamic shared memory of bif_prefix_kernel (the tile ring plus 1 KB for 1024-byte alignment).
+size_t bif_prefix_smem_bytes();
+
+// Raises the kernel's dynamic shared-memory limit on the current device.
+cudaError_t bif_prefix_set_smem_limit();
+
+// Prefix pass: grid (M-tile pairs, prefix chunks, KV heads), one CTA per SM.
+cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensorMap& vmap, const BifParams& p,
+                              cudaStream_t st);
+
+// Merge of the prefix chunks' statistics with the suffix result, per (sample, query head).
+cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,
+                                       const float* out_s, const float* lse_s, float* out, float* lse,
+                                       int n_samples, int n_q_heads, const int* err, cudaStream_t st);
+
+}  // namespace ta

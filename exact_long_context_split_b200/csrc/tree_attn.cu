@@ -10,8 +10,8 @@
 #include <vector>
 
 #include "../../include/tree_attn.h"
-#include "bifurcated_tc.cuh"
-#include "split_kv.cuh"
+#include "bifurcated_tc.h"
+#include "split_kv_instances.h"
 
 namespace ta {
 namespace {
@@ -33,38 +33,14 @@ ta_status cuda_fail(cudaError_t e) {
 // Kernel instances
 // ------------------------------------------------------------------------------------------
 
-struct KernelInfo {
-  void (*fn)(SplitParams);
-  size_t smem;
-  int tile;
-  int threads;
-};
-
-template <typename T, int D, int G, class V>
-KernelInfo make_info() {
-  using C = SplitCfg<T, D, G, V>;
-  return KernelInfo{&split_kv_decode_kernel<T, D, G, V>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
-}
-
-template <typename T, int D, class V>
-bool pick_g(int G, KernelInfo* ki) {
-  switch (G) {
-    case 1: *ki = make_info<T, D, 1, V>(); return true;
-    case 2: *ki = make_info<T, D, 2, V>(); return true;
-    case 4: *ki = make_info<T, D, 4, V>(); return true;
-    case 8: *ki = make_info<T, D, 8, V>(); return true;
-    default: return false;
-  }
-}
-
 template <class V>
 bool pick_variant(ta_dtype dt, int D, int G, KernelInfo* ki) {
   if (dt == TA_BF16) {
-    if (D == 64) return pick_g<__nv_bfloat16, 64, V>(G, ki);
-    if (D == 128) return pick_g<__nv_bfloat16, 128, V>(G, ki);
+    if (D == 64) return split_instance<__nv_bfloat16, V, 64>(G, ki);
+    if (D == 128) return split_instance<__nv_bfloat16, V, 128>(G, ki);
   } else if (dt == TA_F32) {
-    if (D == 64) return pick_g<float, 64, V>(G, ki);
-    if (D == 128) return pick_g<float, 128, V>(G, ki);
+    if (D == 64) return split_instance<float, V, 64>(G, ki);
+    if (D == 128) return split_instance<float, V, 128>(G, ki);
   }
   return false;
 }
@@ -426,8 +402,7 @@ ta_status bif_tc_setup(int* sms) {
   e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
   std::call_once(once, [] {
-    err = cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel),
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sizeof(BifSmem) + 1024));
+    err = bif_prefix_set_smem_limit();
   });
   if (err != cudaSuccess) return cuda_fail(err);
   return TA_OK;
@@ -525,16 +500,13 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
       bpp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
       bpp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
       const dim3 grid(bp.mtiles, bp.chunks, a.Hkv);
-      bif_prefix_kernel<<<grid, kBifThreads, sizeof(BifSmem) + 1024, st>>>(kmap, vmap, bpp);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launch_bif_prefix(grid, kmap, vmap, bpp, st);
       if (e != cudaSuccess) return cuda_fail(e);
       s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                       base + bp.suffix_off, err, st);
       if (s != TA_OK) return s;
-      const int64_t n = static_cast<int64_t>(rows) * (kBifD / 4);  // one thread per 4 columns of a row
-      merge_prefix_suffix_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-          bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse, a.N, a.Hq, err);
-      e = cudaGetLastError();
+      e = launch_merge_prefix_suffix(bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse,
+                                     a.N, a.Hq, err, st);
       if (e != cudaSuccess) return cuda_fail(e);
       return TA_OK;
     }
