@@ -17,6 +17,7 @@ from .attention import (  # noqa: F401
     finalize,
     merge,
     merge_tree,
+    multi_query_attention,
     online_softmax,
     sequence_block,
     split_attention,

@@ -40,6 +40,12 @@ design notes):
 5. GQA: query head h reads KV head h // (Hq / Hkv) (consecutive groups).
 6. The bifurcated result for sample n is plain attention over the concatenation
    [prefix ; suffix_n]; no mask (the query is the last position).
+7. Several query tokens per sequence ([StarAttn], "How Star Attention cuts the cost of
+   inference" and phase 2): a short query of n tokens follows the cached context, and its
+   tokens' keys and values are written to the cache at its end before attention.  Query
+   token j (0-based) sits at position S - n + j and attends to every key at or before it,
+   i.e. to the first S - n + j + 1 keys (all preceding context, causal among the n new
+   tokens).  n = 1 is ordinary decode.
 """
 from __future__ import annotations
 
@@ -289,4 +295,42 @@ def bifurcated_attention(q, k_prefix, v_prefix, prefix_len: int, k_suffix, v_suf
             K = np.concatenate([Kp[g], Ks[g]], axis=0)
             V = np.concatenate([Vp[g], Vs[g]], axis=0)
             out[n, h], lse[n, h] = attention_one(qf[n, h], K, V, scale)
+    return out, lse
+
+
+def multi_query_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_queries: int, n_q_heads: int,
+                          n_kv_heads: int, head_dim: int, scale: float, dtype: str = "bf16",
+                          rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """n query tokens per sequence, causal among themselves (reading 7).
+
+    q: [B][n][Hq][D] (storage format); k_cache, v_cache packed as for decode_attention, each
+    sequence's block already holding the n query tokens' keys and values as its last n rows.
+    Row (b, j, h) is attention over the first S_b - n + j + 1 keys of KV head h // G.
+
+    Returns (out [B][n][Hq][D], lse [B][n][Hq]) in float64.  With `rows`, only those
+    (b, j, h) entries are computed; the rest are NaN.
+    """
+    B, n = len(seqlens), n_queries
+    Hq, Hkv, D = n_q_heads, n_kv_heads, head_dim
+    if Hq % Hkv != 0:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    if n < 1 or any(int(S) < n for S in seqlens):
+        raise ValueError("every sequence must hold its n query tokens")
+    G = Hq // Hkv
+    qf = to_f64(np.asarray(q).reshape(B, n, Hq, D), dtype)
+    out = np.full((B, n, Hq, D), np.nan)
+    lse = np.full((B, n, Hq), np.nan)
+    todo = sorted(set(rows)) if rows is not None else [(b, j, h) for b in range(B) for j in range(n)
+                                                         for h in range(Hq)]
+    for b in sorted({r[0] for r in todo}):
+        Kb = sequence_block(k_cache, seqlens, b, Hkv, D)
+        Vb = sequence_block(v_cache, seqlens, b, Hkv, D)
+        S = int(seqlens[b])
+        for (bb, j, h) in todo:
+            if bb != b:
+                continue
+            visible = S - n + j + 1
+            g = h // G
+            out[b, j, h], lse[b, j, h] = attention_one_bf16_cache(qf[b, j, h], Kb[g][:visible], Vb[g][:visible],
+                                                                  scale, dtype)
     return out, lse

@@ -398,6 +398,59 @@ def pin_long_cache_pieces(O):
         mod.ROWS_PER_PIECE = saved
 
 
+def pin_multi_query(O):
+    """[StarAttn] query tokens attend to all preceding context (reading 7).  (i) A masked score
+    matrix built independently (the n x S scores of all query tokens with -inf above the
+    staircase from np.triu, row softmax by exp / sum) gives every row; (ii) with identical keys
+    query j's out is the mean of its S - n + j + 1 visible value rows and lse = s q.k + ln of
+    that count; (iii) one query per sequence is plain decode of the whole cache."""
+    r = _rng(21)
+    D, Hkv, Hq, n = 4, 2, 4, 3
+    seqlens = [3, 7, 5]
+    G = Hq // Hkv
+    B = len(seqlens)
+    kb = [r.standard_normal((Hkv, S, D)) for S in seqlens]
+    vb = [r.standard_normal((Hkv, S, D)) for S in seqlens]
+    k = np.concatenate([x.reshape(-1) for x in kb])
+    v = np.concatenate([x.reshape(-1) for x in vb])
+    q = r.standard_normal((B, n, Hq, D))
+    out, lse = O.multi_query_attention(q, k, v, seqlens, n, Hq, Hkv, D, 0.7, dtype="f64")
+    for b, S in enumerate(seqlens):
+        # query token j is cache position S - n + j; key t is hidden from it when t > S - n + j
+        hidden = np.triu(np.ones((n, S), dtype=bool), k=S - n + 1)
+        for h in range(Hq):
+            g = h // G
+            X = 0.7 * (q[b, :, h, :] @ kb[b][g].T)
+            X[hidden] = -np.inf
+            mx = X.max(axis=1, keepdims=True)
+            E = np.exp(X - mx)
+            L = E.sum(axis=1)
+            want = (E @ vb[b][g]) / L[:, None]
+            _close(out[b, :, h], want, rtol=1e-12, atol=1e-14, what=f"multi-query rows {b},{h}")
+            _close(lse[b, :, h], mx[:, 0] + np.log(L), rtol=1e-13, what=f"multi-query lse {b},{h}")
+    # (ii) identical keys: the visible count decides both outputs
+    kc = r.standard_normal(D)
+    k_same = np.concatenate([np.tile(kc, (Hkv, S, 1)).reshape(-1) for S in seqlens])
+    out, lse = O.multi_query_attention(q, k_same, v, seqlens, n, Hq, Hkv, D, 0.7, dtype="f64")
+    for b, S in enumerate(seqlens):
+        for j in range(n):
+            cnt = S - n + j + 1
+            for h in range(Hq):
+                g = h // G
+                _close(out[b, j, h], vb[b][g][:cnt].mean(axis=0), rtol=1e-12, atol=1e-14,
+                       what=f"multi-query mean {b},{j},{h}")
+                _close(lse[b, j, h], 0.7 * float(q[b, j, h] @ kc) + math.log(cnt), rtol=1e-13,
+                       what="multi-query lse count")
+    # (iii) n = 1 over the whole cache, against the textbook formula
+    out1, lse1 = O.multi_query_attention(q[:, :1], k, v, seqlens, 1, Hq, Hkv, D, 0.7, dtype="f64")
+    for b, S in enumerate(seqlens):
+        for h in range(Hq):
+            x = 0.7 * (kb[b][h // G] @ q[b, 0, h])
+            e = np.exp(x - x.max())
+            _close(out1[b, 0, h], (e @ vb[b][h // G]) / e.sum(), rtol=1e-12, atol=1e-14, what="n = 1")
+            _close(lse1[b, 0, h], x.max() + math.log(e.sum()), rtol=1e-13, what="n = 1 lse")
+
+
 ALL_PINS = [
     pin_bf16_decoding,
     pin_identical_keys,
@@ -417,4 +470,5 @@ ALL_PINS = [
     pin_packed_layout,
     pin_bifurcated,
     pin_long_cache_pieces,
+    pin_multi_query,
 ]
