@@ -194,7 +194,8 @@ def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra
         "data": "synthetic",
         "config": {
             "workload": spec.name,
-            **({"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0}
+            **({"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
+                "query_tokens": spec.n_queries}
                if isinstance(spec, synth.DecodeSpec) else
                {"samples": spec.n_samples, "prefix_len": spec.prefix_len,
                 "suffix_len": int(max(spec.suffix_lens)) if spec.suffix_lens else 0}),
@@ -309,6 +310,34 @@ class DecodeRun:
                                     stream=stream)
 
 
+class MultiRun(DecodeRun):
+    """Several query tokens per sequence: one call = ceil(n / n') passes of G n' rows per KV head."""
+
+    def __init__(self, spec, torch, ta):
+        super().__init__(spec, torch, ta)
+        B, n, Hq, Hkv, D = spec.batch, spec.n_queries, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+        self.out = torch.empty(B, n, Hq, D, device="cuda")
+        self.lse = torch.empty(B, n, Hq, device="cuda")
+        self.ws = torch.empty(ta.tree_attn_multi_workspace_size(self.seqlens, n, Hq, Hkv, D), dtype=torch.uint8,
+                              device="cuda")
+        ta.tree_attn_workspace_init(self.ws)
+        G, passes, j = Hq // Hkv, 0, 0
+        while j < n:
+            step = 1
+            while 2 * step <= n - j and 2 * step * G <= 8:
+                step *= 2
+            j += step
+            passes += 1
+        self.launches_per_step = passes
+        self.kernel = f"split_kv_decode_kernel<bf16,{D},G*n'> x {passes} passes"
+
+    def step(self, stream):
+        sp = self.spec
+        self.ta.tree_attn_decode_multi_ex("bf16", self.dev["q"], self.dev["k"], self.dev["v"], self.seqlens,
+                                          sp.n_queries, sp.n_q_heads, sp.n_kv_heads, sp.head_dim, sp.scale, self.out,
+                                          self.lse, None, self.ws, stream=stream)
+
+
 class BifurcatedRun:
     """Shared-prefix workload: one call = prefix pass, suffix pass and the exact merge."""
 
@@ -354,7 +383,12 @@ def run_gpu(args, spec) -> None:
                                 device_id=torch.device("cuda", local_rank))
     import exact_long_context_split_b200 as ta
 
-    run = (BifurcatedRun if isinstance(spec, synth.BifurcatedSpec) else DecodeRun)(spec, torch, ta)
+    if isinstance(spec, synth.BifurcatedSpec):
+        run = BifurcatedRun(spec, torch, ta)
+    elif spec.n_queries > 1:
+        run = MultiRun(spec, torch, ta)
+    else:
+        run = DecodeRun(spec, torch, ta)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
@@ -422,13 +456,13 @@ def run_gpu(args, spec) -> None:
         "gpu_launches": args.steps * run.launches_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_kind": peak_kind, "kernel": run.kernel,
-                     "traffic": traffic_per_launch(spec) if isinstance(run, DecodeRun) else None},
+                     "traffic": traffic_per_launch(spec) if type(run) is DecodeRun else None},
         "clocks": clocks.summary(),
     }
     if isinstance(run, BifurcatedRun):
         extra["logical_kv_tokens_per_s"] = world * spec.n_samples * (spec.prefix_len + statistics.mean(run.lens)) * \
             args.steps / (elapsed_ms * 1e-3)
-    if world == 1 and not args.no_cpu_baseline and isinstance(run, DecodeRun):
+    if world == 1 and not args.no_cpu_baseline and type(run) is DecodeRun:
         G = spec.n_q_heads // spec.n_kv_heads
         sec = oracle_sample_seconds(spec, 0, list(range(G)))
         rows = spec.batch * spec.n_q_heads
@@ -452,7 +486,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    workloads = {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs()}
+    workloads = {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs(),
+                 **synth.multi_query_configs()}
     ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

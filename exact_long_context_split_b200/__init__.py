@@ -32,6 +32,9 @@ EXPORTED = [
     "tree_attn_decode_bifurcated_ex",
     "tree_attn_check",
     "tree_attn_decode_noalloc",
+    "tree_attn_multi_workspace_size",
+    "tree_attn_decode_multi_ex",
+    "tree_attn_decode_multi",
 ]
 
 
@@ -102,6 +105,12 @@ def lib() -> ctypes.CDLL:
             ),
             "tree_attn_check": ([vp, vp], ctypes.c_int),
             "tree_attn_decode_noalloc": ([vp, vp, vp, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
+            "tree_attn_multi_workspace_size": ([pi64, i32, i32, i32, i32, i32, ctypes.c_int, popt, psz], ctypes.c_int),
+            "tree_attn_decode_multi_ex": (
+                [ctypes.c_int, vp, vp, vp, pi64, i32, i32, i32, i32, i32, f32, vp, vp, popt, vp, sz, vp],
+                ctypes.c_int,
+            ),
+            "tree_attn_decode_multi": ([vp, vp, vp, pi64, i32, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -243,3 +252,33 @@ def tree_attn_decode_noalloc(q, k_cache, v_cache, seqlens, n_q_heads, n_kv_heads
     _check(lib().tree_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), arr, n, n_q_heads, n_kv_heads,
                                           head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
            "tree_attn_decode_noalloc")
+
+
+def tree_attn_multi_workspace_size(seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, dtype="bf16",
+                                   opts=None) -> int:
+    arr, n = _lens(seqlens)
+    out = ctypes.c_size_t(0)
+    _check(lib().tree_attn_multi_workspace_size(arr, n, n_queries, n_q_heads, n_kv_heads, head_dim, _DTYPES[dtype],
+                                                _opts(opts), ctypes.byref(out)), "tree_attn_multi_workspace_size")
+    return out.value
+
+
+def tree_attn_decode_multi_ex(dtype, q, k_cache, v_cache, seqlens, n_queries, n_q_heads, n_kv_heads, head_dim,
+                              scale, out, lse, opts, workspace, workspace_bytes: Optional[int] = None,
+                              stream=None) -> None:
+    """n query tokens per sequence, causal among themselves: q, out [B][n][Hq][D], lse [B][n][Hq]."""
+    arr, n = _lens(seqlens)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().tree_attn_decode_multi_ex(_DTYPES[dtype], _ptr(q), _ptr(k_cache), _ptr(v_cache), arr, n, n_queries,
+                                           n_q_heads, n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse), _opts(opts),
+                                           _ptr(workspace), workspace_bytes, _stream(stream, q, out)),
+           "tree_attn_decode_multi_ex")
+
+
+def tree_attn_decode_multi(q, k_cache, v_cache, seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, scale, out,
+                           lse, stream=None) -> None:
+    arr, n = _lens(seqlens)
+    _check(lib().tree_attn_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), arr, n, n_queries, n_q_heads,
+                                        n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
+           "tree_attn_decode_multi")

@@ -305,7 +305,8 @@ __device__ __forceinline__ void bif_exp_chunk(const float (&x)[32], uint32_t col
   for (int c2 = 0; c2 < 16; ++c2) {
     const float2 y = __ffma2_rn(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, nm);
     float2 pp;
-    if (kBifPolyEvery > 0 && c2 % kBifPolyEvery == kBifPolyEvery - 1)
+    constexpr int kMod = kBifPolyEvery > 0 ? kBifPolyEvery : 1;
+    if (kBifPolyEvery > 0 && c2 % kMod == kMod - 1)
       pp = exp2_poly2(y);
     else
       pp = make_float2(ex2(y.x), ex2(y.y));
@@ -682,13 +683,13 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 // ---------------------------------------------------------------------------------------------
 
 // Suffix part given normalised (out_s, lse_s); it enters as m = lse_s log2(e), l = 1, o = out_s.
-// One thread per 4 columns of an output row; the chunk loops are unrolled so that the
-// partials' loads are in flight together.
-__global__ void merge_prefix_suffix_kernel(const float* __restrict__ part, int n_chunks, int n_kv_heads,
-                                           int rows_per_head, const float* __restrict__ out_s,
-                                           const float* __restrict__ lse_s, float* __restrict__ out,
-                                           float* __restrict__ lse, int n_samples, int n_q_heads,
-                                           const int* __restrict__ err) {
+// One thread per 4 columns of an output row.  One online pass over the chunks (the running
+// max moves only when a chunk's m exceeds it): each chunk's loads depend on nothing computed
+// before them, so an unrolled group of chunks has all its loads in flight at once.
+__global__ void __launch_bounds__(128) merge_prefix_suffix_kernel(
+    const float* __restrict__ part, int n_chunks, int n_kv_heads, int rows_per_head, const float* __restrict__ out_s,
+    const float* __restrict__ lse_s, float* __restrict__ out, float* __restrict__ lse, int n_samples, int n_q_heads,
+    const int* __restrict__ err) {
   constexpr int Q = kBifD / 4;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total = static_cast<int64_t>(n_samples) * n_q_heads * Q;
@@ -701,32 +702,22 @@ __global__ void merge_prefix_suffix_kernel(const float* __restrict__ part, int n
   const float* base = part + (static_cast<int64_t>(h) * rows_per_head + n * G + g) * kBifPartRow;
   const int64_t stride = static_cast<int64_t>(n_kv_heads) * rows_per_head * kBifPartRow;
   const float ls = lse_s[rq];
-  const float ms = (ls == -INFINITY) ? -INFINITY : ls * 1.44269504088896340736f;
-  float M = ms;
-#pragma unroll 8
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, base[c * stride]);
-  float L = 0.f;
-  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-#pragma unroll 8
-    for (int c = 0; c < n_chunks; ++c) {
-      const float* pc = base + c * stride;
-      const float2 ml = *reinterpret_cast<const float2*>(pc);
-      const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
-      const float w = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - M);
-      L += w * ml.y;
-      O.x += w * o.x;
-      O.y += w * o.y;
-      O.z += w * o.z;
-      O.w += w * o.w;
-    }
-    const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-    const float4 os = *reinterpret_cast<const float4*>(out_s + rq * kBifD + d4);
-    L += w;
-    O.x += w * os.x;
-    O.y += w * os.y;
-    O.z += w * os.z;
-    O.w += w * os.w;
+  float M = (ls == -INFINITY) ? -INFINITY : ls * 1.44269504088896340736f;
+  float L = (ls == -INFINITY) ? 0.f : 1.f;
+  float4 O = (ls == -INFINITY) ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : *reinterpret_cast<const float4*>(out_s + rq * kBifD + d4);
+#pragma unroll 9
+  for (int c = 0; c < n_chunks; ++c) {
+    const float* pc = base + c * stride;
+    const float2 ml = *reinterpret_cast<const float2*>(pc);
+    const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
+    if (ml.x == -INFINITY) continue;  // empty chunk
+    const float Mn = fmaxf(M, ml.x);
+    const float a = (M == -INFINITY) ? 0.f : ex2(M - Mn);
+    const float b = ex2(ml.x - Mn);
+    L = L * a + ml.y * b;
+    O = make_float4(O.x * a + o.x * b, O.y * a + o.y * b, O.z * a + o.z * b, O.w * a + o.w * b);
+    M = Mn;
   }
   float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
   float lv = -INFINITY;

@@ -57,11 +57,19 @@ struct SplitParams {
   float scale_log2;       // scale * log2(e): scores come out in base-2 units
   int32_t debug_skip_tile;
   int32_t unit_aligned;   // 1: CTA ranges start at unit boundaries, so no unit is shared by CTAs
+  // Several query tokens per sequence: q is [B][n_queries][Hq][D] (out and lse alike) and the
+  // G rows of a unit are query tokens q_first + r / heads, query heads h * heads + r % heads,
+  // heads = 1 << log2_heads; query token j sees the first S - n_queries + j + 1 keys.  Plain
+  // decode: n_queries = 1, q_first = 0, heads = G.
+  int32_t n_queries;
+  int32_t q_first;
+  int32_t log2_heads;
   int64_t kv_off[kMaxSeqPerLaunch];
   int64_t seq_len[kMaxSeqPerLaunch];
   int64_t tile_off[kMaxSeqPerLaunch + 1];  // first tile of sequence b on the line
   int32_t n_tiles[kMaxSeqPerLaunch];       // tiles per (sequence, KV head), >= 1
 };
+static_assert(sizeof(SplitParams) <= 4096, "kernel parameters must fit the 4 KB parameter space");
 
 // Tile configurations of the split kernel (measured on B200; see the design notes).
 // LongTiles: 12 consumer warps, 8 row elements per lane, 48 KB K and V tiles, a 2-deep ring:
@@ -340,8 +348,8 @@ __device__ __forceinline__ float tree_sum(const float (&a)[M]) {
 // out = O / L, lse = ln(2) (M + log2 L); an empty unit gives 0 and -inf; a unit whose
 // inputs may be incomplete (this CTA gave up waiting: `poisoned`) gives NaN.  NaN partials
 // of another CTA propagate through the merge weights (2^(NaN - M) is NaN).
-__device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq, int d, int D, float M, float L,
-                                            float O, bool write_lse, bool poisoned) {
+__device__ __forceinline__ void write_final(const SplitParams& p, int b, int h, int r, int d, int D, float M,
+                                            float L, float O, bool write_lse, bool poisoned) {
   float ov, lv;
   if (L > 0.f) {
     ov = O / L;
@@ -354,7 +362,8 @@ __device__ __forceinline__ void write_final(const SplitParams& p, int b, int hq,
     ov = __int_as_float(0x7fc00000);
     lv = ov;
   }
-  const int64_t row = static_cast<int64_t>(b) * p.n_q_heads + hq;
+  const int64_t row = (static_cast<int64_t>(b) * p.n_queries + p.q_first + (r >> p.log2_heads)) * p.n_q_heads +
+                      (h << p.log2_heads) + (r & ((1 << p.log2_heads) - 1));
   p.out[row * D + d] = ov;
   if (write_lse) p.lse[row] = lv;
 }
@@ -421,9 +430,16 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
           uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
           mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
           if (with_q) {
-            const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
-                                  (static_cast<int64_t>(w.b) * p.n_q_heads + w.h * G) * D * C::ELEM;
-            bulk_load(sm.q[s], qsrc, q_bytes, &sm.full[s], pol);
+            // One copy per query token of the launch: its `heads` query heads are contiguous.
+            const int heads = 1 << p.log2_heads;
+            const uint32_t qb = static_cast<uint32_t>(heads) * D * C::ELEM;
+            for (int jl = 0; jl < (G >> p.log2_heads); ++jl) {
+              const uint8_t* qsrc =
+                  reinterpret_cast<const uint8_t*>(p.q) +
+                  ((static_cast<int64_t>(w.b) * p.n_queries + p.q_first + jl) * p.n_q_heads + w.h * heads) * D *
+                      C::ELEM;
+              bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
+            }
           }
           if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
           if (bytes != 0) {
@@ -464,6 +480,9 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
     float2 q2[G][E2];  // q * scale * log2(e), the G heads of the current KV head
     float2 o2[G][E2];  // unnormalised output of this lane's tokens
     float m = -INFINITY, l = 0.f;  // statistics of head head_of_lane(li) over this lane's tokens
+    // Keys at the end of the sequence this lane's row may not see: query token j of n is
+    // n - 1 - j positions before the last one (0 for plain decode).
+    const int lag = p.n_queries - 1 - (p.q_first + (head_of_lane<G, C::LPT>(li) >> p.log2_heads));
 
     // The unit's q (landed in stage s with the unit's first tile), read like a K row so the
     // register order matches the K elements it multiplies.
@@ -550,7 +569,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
           }
           const float O = tree_sum<C::NCW>(ao), L = tree_sum<C::NCW>(al);
           if (n_parts == 1) {
-            write_final(p, b, h * G + g, d, D, Mx, L, O, d == 0, poisoned);
+            write_final(p, b, h, g, d, D, Mx, L, O, d == 0, poisoned);
           } else {
             const float nan = __int_as_float(0x7fc00000);
             slot[2 * G + g * D + d] = poisoned ? nan : O;
@@ -628,7 +647,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
             const int col = tid + k * C::NCT;
             if (col < G * D) {
               const int g = col / D, d = col % D;
-              write_final(p, b, h * G + g, d, D, sm.mM[g], sm.mL[g], acc[k].result(), d == 0, poisoned);
+              write_final(p, b, h, g, d, D, sm.mM[g], sm.mL[g], acc[k].result(), d == 0, poisoned);
             }
           }
           if (tid == 0) p.tickets[unit] = 0;
@@ -666,6 +685,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
       if (ok) {
         const int64_t len = p.seq_len[w.b];
         const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - w.j * C::TILE));
+        const int nv_row = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - lag - w.j * C::TILE));
         const uint8_t* kt = sm.k[s];
         const uint8_t* vt = sm.v[s];
         // Phase A: the scores of this warp's STEPS tokens of the tile (independent chains).
@@ -684,7 +704,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
             sc[g] = acc.x + acc.y;
           }
           const float xs = reduce_scores<G, C::LPT>(sc, li);
-          x[st] = (tok < nv) ? xs : -INFINITY;
+          x[st] = (tok < nv_row) ? xs : -INFINITY;
         }
         // Phase B: one online-softmax update for the tile (lazy rescaling of m).
         float xm = x[0];

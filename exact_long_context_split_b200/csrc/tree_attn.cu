@@ -205,19 +205,25 @@ bool any_tokens(const int64_t* seqlens, int batch) {
 // Launch of a planned decode (workspace body at `body`, error word at `err`)
 // ------------------------------------------------------------------------------------------
 
+// n_queries / q_first: query tokens per sequence and the first one this launch covers (the
+// kernel instance's G rows per unit are G / (Hq / Hkv) consecutive query tokens).
 ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, const void* k, const void* v,
                       float* out, float* lse, int Hq, int Hkv, int D, float scale, ta_dtype dt,
-                      const ta_options* opts, uint8_t* body, int* err, cudaStream_t st) {
+                      const ta_options* opts, uint8_t* body, int* err, cudaStream_t st, int n_queries = 1,
+                      int q_first = 0) {
   const size_t qe = (dt == TA_BF16) ? 2 : 4;
+  int log2_heads = 0;
+  while ((1 << (log2_heads + 1)) <= Hq / Hkv) ++log2_heads;
   const double s2 = static_cast<double>(scale) * 1.4426950408889634073599246810019;
   for (const Group& g : plan.groups) {
     SplitParams p;
     std::memset(&p, 0, sizeof(p));
-    p.q = static_cast<const uint8_t*>(q) + static_cast<size_t>(g.b0) * Hq * D * qe;
+    const size_t rows0 = static_cast<size_t>(g.b0) * n_queries * Hq;  // first output row of the group
+    p.q = static_cast<const uint8_t*>(q) + rows0 * D * qe;
     p.k = k;
     p.v = v;
-    p.out = out + static_cast<size_t>(g.b0) * Hq * D;
-    p.lse = lse + static_cast<size_t>(g.b0) * Hq;
+    p.out = out + rows0 * D;
+    p.lse = lse + rows0;
     p.tickets = reinterpret_cast<int*>(body + g.tickets_off);
     p.part = reinterpret_cast<float*>(body + g.part_off);
     p.err = err;
@@ -230,6 +236,9 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
     p.scale_log2 = static_cast<float>(s2);
     p.debug_skip_tile = opts ? opts->debug_skip_tile : -1;
     p.unit_aligned = g.unit_aligned ? 1 : 0;
+    p.n_queries = n_queries;
+    p.q_first = q_first;
+    p.log2_heads = log2_heads;
     for (int i = 0; i < g.nb; ++i) {
       p.kv_off[i] = g.kv_off[i];
       p.seq_len[i] = g.len[i];
@@ -308,6 +317,68 @@ ta_status with_temp_workspace(size_t bytes, cudaStream_t st, ta_status (*run)(vo
   e = cudaFreeAsync(ws, st);
   if (s != TA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e);
+  return TA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Several query tokens per sequence: passes of G * n' rows per unit (n' query tokens, a power
+// of two with G * n' <= 8), each over the whole cache, sharing one workspace in turn.
+// ------------------------------------------------------------------------------------------
+
+struct MultiPass {
+  int q_first = 0, n_q = 0;
+  KernelInfo ki;
+  Plan plan;
+};
+
+ta_status multi_validate(const DecodeArgs& a, int n_queries, const ta_options* opts, bool check_pointers,
+                         KernelInfo* ki) {
+  if (n_queries < 1) return TA_ERR_INVALID_ARG;
+  const ta_status s = validate(a, opts, check_pointers, ki);
+  if (s != TA_OK) return s;
+  for (int b = 0; b < a.batch; ++b)
+    if (a.seqlens[b] < n_queries) return TA_ERR_INVALID_ARG;  // the query tokens are in the cache
+  return TA_OK;
+}
+
+ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts, std::vector<MultiPass>* passes,
+                     size_t* body_max) {
+  const int G = a.Hq / a.Hkv;
+  const bool short_tiles = use_short_tiles(a.seqlens, a.batch, opts);
+  passes->clear();
+  *body_max = 0;
+  for (int j0 = 0; j0 < n_queries;) {
+    int nq = 1;
+    while (2 * nq <= n_queries - j0 && G * 2 * nq <= 8) nq *= 2;
+    MultiPass mp;
+    mp.q_first = j0;
+    mp.n_q = nq;
+    if (!pick_kernel(a.dt, a.D, G * nq, short_tiles, &mp.ki)) return TA_ERR_UNSUPPORTED;
+    int dev = 0, slots = 1;
+    if (a.batch > 0) {
+      const ta_status s = resident_ctas(mp.ki, &dev, &slots);
+      if (s != TA_OK) return s;
+    }
+    const ta_status s = build_plan(a.seqlens, a.kv_offsets, a.batch, a.Hkv, G * nq, a.D, mp.ki.tile, slots, opts,
+                                   &mp.plan);
+    if (s != TA_OK) return s;
+    *body_max = std::max(*body_max, mp.plan.body_bytes);
+    passes->push_back(mp);
+    j0 += nq;
+  }
+  return TA_OK;
+}
+
+ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, const std::vector<MultiPass>& passes,
+                    void* ws, size_t ws_bytes, size_t body_max, cudaStream_t st) {
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < kHeaderBytes + body_max) return TA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  for (const MultiPass& mp : passes) {
+    const ta_status s = launch_plan(mp.plan, mp.ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt,
+                                    opts, base + kHeaderBytes, reinterpret_cast<int*>(base), st, n_queries,
+                                    mp.q_first);
+    if (s != TA_OK) return s;
+  }
   return TA_OK;
 }
 
@@ -674,6 +745,69 @@ ta_status tree_attn_decode_bifurcated(const void* q, const void* k_prefix, const
   if (s != TA_OK) return s;
   BifCtx ctx{a, &bp};
   return with_temp_workspace(bp.total, static_cast<cudaStream_t>(stream), &bif_alloc_run, &ctx);
+}
+
+ta_status tree_attn_multi_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_queries,
+                                         int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, ta_dtype dtype,
+                                         const ta_options* opts, size_t* bytes) {
+  if (!bytes) return TA_ERR_INVALID_ARG;
+  DecodeArgs a{dtype, nullptr, nullptr, nullptr, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               1.0f, nullptr, nullptr};
+  KernelInfo ki;
+  ta_status s = multi_validate(a, n_queries, opts, false, &ki);
+  if (s != TA_OK) return s;
+  std::vector<MultiPass> passes;
+  size_t body = 0;
+  s = multi_plan(a, n_queries, opts, &passes, &body);
+  if (s != TA_OK) return s;
+  *bytes = kHeaderBytes + body;
+  return TA_OK;
+}
+
+ta_status tree_attn_decode_multi_ex(ta_dtype dtype, const void* q, const void* k_cache, const void* v_cache,
+                                    const int64_t* seqlens, int32_t batch, int32_t n_queries, int32_t n_q_heads,
+                                    int32_t n_kv_heads, int32_t head_dim, float scale, float* out, float* lse,
+                                    const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  DecodeArgs a{dtype, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  KernelInfo ki;
+  ta_status s = multi_validate(a, n_queries, opts, true, &ki);
+  if (s != TA_OK || batch == 0) return s;
+  std::vector<MultiPass> passes;
+  size_t body = 0;
+  s = multi_plan(a, n_queries, opts, &passes, &body);
+  if (s != TA_OK) return s;
+  return multi_run(a, n_queries, opts, passes, workspace, workspace_bytes, body, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+struct MultiCtx {
+  DecodeArgs a;
+  int n_queries;
+  const std::vector<MultiPass>* passes;
+  size_t body;
+};
+ta_status multi_alloc_run(void* ws, size_t bytes, void* ctx, cudaStream_t st) {
+  MultiCtx* c = static_cast<MultiCtx*>(ctx);
+  return multi_run(c->a, c->n_queries, nullptr, *c->passes, ws, bytes, c->body, st);
+}
+}  // namespace
+
+ta_status tree_attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                                 int32_t batch, int32_t n_queries, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int32_t head_dim, float scale, float* out, float* lse, void* stream) {
+  DecodeArgs a{TA_BF16, q, k_cache, v_cache, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  KernelInfo ki;
+  ta_status s = multi_validate(a, n_queries, nullptr, true, &ki);
+  if (s != TA_OK || batch == 0) return s;
+  std::vector<MultiPass> passes;
+  size_t body = 0;
+  s = multi_plan(a, n_queries, nullptr, &passes, &body);
+  if (s != TA_OK) return s;
+  MultiCtx ctx{a, n_queries, &passes, body};
+  return with_temp_workspace(kHeaderBytes + body, static_cast<cudaStream_t>(stream), &multi_alloc_run, &ctx);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -136,6 +136,36 @@ ta_status tree_attn_decode_ex(ta_dtype dtype, const void* q, const void* k_cache
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Several query tokens per sequence (speculative or multi-token decode), after the Star
+ * Attention article (tiaojiaomugou.com, "How Star Attention cuts the cost of inference" and
+ * "Phase 2: query encoding and token generation"): a short query of n tokens follows the
+ * cached context, with the tokens' keys and values already written as the last n rows of each
+ * sequence's cache, and each query token attends to all the context before it and to itself.
+ * Query token j (0-based) of sequence b sits at position S_b - n + j and attends to the first
+ * S_b - n + j + 1 keys (causal among the n new tokens).  n = 1 is tree_attn_decode.
+ *   q    [B][n][Hq][D]  bf16 (or f32 with TA_F32)
+ *   k, v packed per sequence as for tree_attn_decode; every S_b >= n, else TA_ERR_INVALID_ARG
+ *   out  [B][n][Hq][D]  f32;  lse [B][n][Hq] f32
+ * One pass over the cache serves G * n' rows per KV head (n' consecutive query tokens, a power
+ * of two, G * n' <= 8, G = n_q_heads / n_kv_heads); larger n takes several passes, run in turn
+ * on `stream` with one workspace.  Other rules as tree_attn_decode / tree_attn_decode_ex.
+ */
+ta_status tree_attn_multi_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_queries,
+                                         int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, ta_dtype dtype,
+                                         const ta_options* opts, size_t* bytes);
+
+/* Multi-query decode with a caller-owned, zero-filled workspace (rules as tree_attn_decode_ex). */
+ta_status tree_attn_decode_multi_ex(ta_dtype dtype, const void* q, const void* k_cache, const void* v_cache,
+                                    const int64_t* seqlens, int32_t batch, int32_t n_queries, int32_t n_q_heads,
+                                    int32_t n_kv_heads, int32_t head_dim, float scale, float* out, float* lse,
+                                    const ta_options* opts, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Multi-query decode, bf16, allocating its workspace per call like tree_attn_decode. */
+ta_status tree_attn_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
+                                 int32_t batch, int32_t n_queries, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int32_t head_dim, float scale, float* out, float* lse, void* stream);
+
+/*
  * Bifurcated (shared-prefix) decode, after the bifurcated-attention summary
  * (briefgpt.xyz, 2403.08845, TL;DR): sample n's query attends over the
  * concatenation [prefix ; suffix_n] — one shared context prefilled once plus the

@@ -112,7 +112,8 @@ def bf16_bits_from_f32(a: np.ndarray) -> np.ndarray:
 
 @dataclasses.dataclass(frozen=True)
 class DecodeSpec:
-    """One decode step: B sequences, one query token per (sequence, query head)."""
+    """One decode step: B sequences, n_queries query tokens per (sequence, query head) (the
+    last n_queries cache rows are those tokens' keys and values)."""
 
     name: str
     seqlens: Sequence[int]
@@ -124,6 +125,7 @@ class DecodeSpec:
     spike_frac: float = 0.0  # fraction of keys per KV head scaled by spike_factor
     spike_factor: float = 4.0
     scale_value: Optional[float] = None  # softmax scale; default 1/sqrt(head_dim) rounded to float32
+    n_queries: int = 1
 
     @property
     def batch(self) -> int:
@@ -193,6 +195,15 @@ def decode_configs() -> Dict[str, DecodeSpec]:
     }
 
 
+def multi_query_configs() -> Dict[str, DecodeSpec]:
+    """Several query tokens per sequence (speculative decode verifying draft tokens): the
+    32K x 8 batch of llama3_8b_gqa with 2 and with 4 query tokens per sequence."""
+    return {
+        "spec_decode_2": DecodeSpec("spec_decode_2", [32768] * 8, 32, 8, 128, seed=7, n_queries=2),
+        "spec_decode_4": DecodeSpec("spec_decode_4", [32768] * 8, 32, 8, 128, seed=8, n_queries=4),
+    }
+
+
 def capture_configs() -> Dict[str, DecodeSpec]:
     """Smaller versions of the long-context workload for profiler captures (same recipe,
     1/4 of the length: 1.07 GB of K/V, still far larger than the 126 MB L2)."""
@@ -206,7 +217,8 @@ def bifurcated_configs() -> Dict[str, BifurcatedSpec]:
 def make_decode_inputs(spec: DecodeSpec) -> Dict[str, np.ndarray]:
     """Host buffers for one decode step (bf16 as uint16 bits, f32 as float32)."""
     B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
-    nq = B * Hq * D
+    n = spec.n_queries
+    nq = B * n * Hq * D
     if spec.dtype == "bf16":
         q = normal_bf16(spec.seed, TID_Q, nq)
         k = normal_bf16(spec.seed, TID_K, spec.kv_elems)
@@ -228,7 +240,7 @@ def make_decode_inputs(spec: DecodeSpec) -> Dict[str, np.ndarray]:
                 spikes.append(spike_rows_bf16(rows, spec.seed, b * Hkv + h, spec.n_spikes(S), spec.spike_factor))
                 off += S * D
     return {
-        "q": q.reshape(B, Hq, D),
+        "q": q.reshape(B, Hq, D) if n == 1 else q.reshape(B, n, Hq, D),
         "k": k,
         "v": v,
         "seqlens": np.asarray(spec.seqlens, dtype=np.int64),
