@@ -311,7 +311,8 @@ class DecodeRun:
 
 
 class MultiRun(DecodeRun):
-    """Several query tokens per sequence: one call = ceil(n / n') passes of G n' rows per KV head."""
+    """Several query tokens per sequence: one call = the tensor-core form (bf16, D = 128,
+    8 <= G n <= 128) or ceil(n G / 8) split-KV passes."""
 
     def __init__(self, spec, torch, ta):
         super().__init__(spec, torch, ta)
@@ -321,15 +322,23 @@ class MultiRun(DecodeRun):
         self.ws = torch.empty(ta.tree_attn_multi_workspace_size(self.seqlens, n, Hq, Hkv, D), dtype=torch.uint8,
                               device="cuda")
         ta.tree_attn_workspace_init(self.ws)
-        G, passes, j = Hq // Hkv, 0, 0
-        while j < n:
-            step = 1
-            while 2 * step <= n - j and 2 * step * G <= 8:
-                step *= 2
-            j += step
-            passes += 1
-        self.launches_per_step = passes
-        self.kernel = f"split_kv_decode_kernel<bf16,{D},G*n'> x {passes} passes"
+        G = Hq // Hkv
+        if D == 128 and 8 <= G * n <= 128:
+            # tensor-core form (the library's automatic choice for bf16): per group of up to 128
+            # sequences one bif_prefix_kernel launch and one merge_chunks_kernel launch
+            groups = (B + 127) // 128
+            self.launches_per_step = 2 * groups
+            self.kernel = f"bif_prefix_kernel (several query tokens, {G * n} rows per KV head) + merge_chunks_kernel"
+        else:
+            passes, j = 0, 0
+            while j < n:
+                step = 1
+                while 2 * step <= n - j and 2 * step * G <= 8:
+                    step *= 2
+                j += step
+                passes += 1
+            self.launches_per_step = passes
+            self.kernel = f"split_kv_decode_kernel<bf16,{D},G*n'> x {passes} passes"
 
     def step(self, stream):
         sp = self.spec

@@ -16,6 +16,15 @@ cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensor
   return cudaGetLastError();
 }
 
+cudaError_t launch_merge_chunks(const float* part, int n_chunks, int n_kv_heads, int rows_per_head, int n_queries,
+                                float* out, float* lse, int batch, int n_q_heads, const int* err, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(batch) * n_queries * n_q_heads * (kBifD / 4);  // one thread per 4 columns
+  if (n == 0) return cudaSuccess;
+  merge_chunks_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
+      part, n_chunks, n_kv_heads, rows_per_head, n_queries, out, lse, batch, n_q_heads, err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,
                                        const float* out_s, const float* lse_s, float* out, float* lse,
                                        int n_samples, int n_q_heads, const int* err, cudaStream_t st) {

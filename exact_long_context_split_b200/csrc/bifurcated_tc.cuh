@@ -387,10 +387,21 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int chunk = blockIdx.y, h = blockIdx.z;
-  const int row0 = blockIdx.x * kBifMT * kBifRows;  // first row of this CTA in the head's query matrix
-  const int n_mt = min(kBifMT, (p.rows_per_head - row0 + kBifRows - 1) / kBifRows);  // active M tiles
-  const int64_t n_tiles = (p.prefix_len + kBifKeys - 1) / kBifKeys;
+  // The CTA's unit: its rows, its keys (a range of tensor-map rows) and its chunk of them.
+  const bool multi = p.mode == 1;
+  const int chunk = multi ? blockIdx.x : blockIdx.y;
+  const int h = multi ? blockIdx.y : blockIdx.z;
+  const int b = multi ? blockIdx.z : 0;
+  const int row0 = multi ? 0 : blockIdx.x * kBifMT * kBifRows;  // first row of this CTA in the unit
+  // Mode 0: M tile w holds rows row0 + 128 w + lane and reads every key tile.  Mode 1: both
+  // slots hold the unit's rows; slot w reads key tiles w, w + 2, ... ("split" slots).
+  const int n_mt = multi ? 1 : min(kBifMT, (p.rows_per_head - row0 + kBifRows - 1) / kBifRows);
+  const bool split = multi;
+  const int n_slots = split ? kBifMT : n_mt;
+  const int64_t kv_len = multi ? p.kv_len[b] : p.prefix_len;
+  const int64_t kv_row0 = multi ? p.kv_row0[b] + h * kv_len : static_cast<int64_t>(h) * p.prefix_len;
+  const int q_tok0 = multi ? b * p.n_queries : 0;  // q row of the unit's first token / sample
+  const int64_t n_tiles = (kv_len + kBifKeys - 1) / kBifKeys;
   const int64_t j0 = chunk * n_tiles / p.n_chunks;
   const int n_t = static_cast<int>((chunk + 1) * n_tiles / p.n_chunks - j0);
 
@@ -398,13 +409,13 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 #pragma unroll
     for (int s = 0; s < kBifKStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], n_mt);  // one commit per active M tile's S = Q K^T
+      mbar_init(&sm.k_empty[s], split ? 1 : n_mt);  // one commit per S = Q K^T that reads it
     }
 #pragma unroll
     for (int s = 0; s < kBifVStages; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_conv[s], 64);
-      mbar_init(&sm.v_empty[s], n_mt);  // one commit per active M tile's O += P V
+      mbar_init(&sm.v_empty[s], split ? 1 : n_mt);  // one commit per O += P V that reads it
     }
 #pragma unroll
     for (int w = 0; w < kBifMT; ++w) {
@@ -438,7 +449,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       uint64_t pol;
       asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
       auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int t) {
-        const int y = static_cast<int>(h * p.prefix_len + (j0 + t) * kBifKeys);
+        const int y = static_cast<int>(kv_row0 + (j0 + t) * kBifKeys);
         mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
         tma_load_2d(dst, map, 0, y, full, pol);
         tma_load_2d(dst + kBifKeys * 128, map, 64, y, full, pol);
@@ -487,20 +498,22 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       // Per M tile w the stream is S(0), PV(0), S(1), PV(1), ...: S(t + 1) overwrites the
       // TMEM columns where P(t) was read, so it follows P(t) V(t) in issue order.
       int tq[kBifMT] = {0, 0}, tp[kBifMT] = {0, 0};
+      int nw[kBifMT];  // key tiles of each slot; a slot's local tile t is the CTA's tile t or 2 t + w
+      for (int w = 0; w < kBifMT; ++w) nw[w] = w >= n_slots ? 0 : (split ? (n_t - w + 1) / 2 : n_t);
       auto all_done = [&]() {
-        for (int w = 0; w < n_mt; ++w)
-          if (tp[w] < n_t) return false;
+        for (int w = 0; w < n_slots; ++w)
+          if (tp[w] < nw[w]) return false;
         return true;
       };
       uint64_t t_idle = global_timer_ns();
       while (ok && !all_done()) {
         bool progress = false;
-        for (int w = 0; w < n_mt; ++w) {
-          if (tq[w] == tp[w] && tq[w] < n_t) {
-            const int t = tq[w], s = t % kBifKStages;
+        for (int w = 0; w < n_slots; ++w) {
+          if (tq[w] == tp[w] && tq[w] < nw[w]) {
+            const int t = split ? 2 * tq[w] + w : tq[w], s = t % kBifKStages;
             if (mbar_test_wait(&sm.k_full[s], (t / kBifKStages) & 1)) {
               tc_fence_after();
-              const uint32_t q_base = smem_addr(sm.q[w]);
+              const uint32_t q_base = smem_addr(sm.q[split ? 0 : w]);
               const uint32_t k_base = smem_addr(sm.k[s]);
 #pragma unroll
               for (int kk = 0; kk < kBifD / 16; ++kk) {
@@ -515,8 +528,8 @@ __global__ void __launch_bounds__(kBifThreads, 1)
               progress = true;
             }
           } else if (tp[w] < tq[w]) {
-            const int t = tp[w], s = t % kBifVStages;
-            if (mbar_test_wait(&sm.v_conv[s], (t / kBifVStages) & 1) && mbar_test_wait(&sm.p_full[w], t & 1)) {
+            const int t = tp[w], tg = split ? 2 * t + w : t, s = tg % kBifVStages;
+            if (mbar_test_wait(&sm.v_conv[s], (tg / kBifVStages) & 1) && mbar_test_wait(&sm.p_full[w], t & 1)) {
               tc_fence_after();
               const uint32_t v_base = smem_addr(sm.v[s]);
 #pragma unroll
@@ -525,7 +538,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
                 tc_mma_f16_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, bd, idesc_pv, t > 0 || kk > 0);
               }
               tc_commit(&sm.v_empty[s]);
-              if (t == n_t - 1) tc_commit(&sm.o_done[w]);
+              if (t == nw[w] - 1) tc_commit(&sm.o_done[w]);
               ++tp[w];
               progress = true;
             }
@@ -576,39 +589,47 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     const uint32_t s_col = tmem + lane_base + w * 128;
     const uint32_t o_col = tmem + lane_base + 256 + w * 128;
     const int G = p.n_q_heads / p.n_kv_heads;
-    const int row = row0 + w * kBifRows + r;          // row of this KV head's query matrix
+    const int row = split ? r : row0 + w * kBifRows + r;  // row of the unit's query matrix
     const bool valid_row = row < p.rows_per_head;
-    {
+    // Keys at the end of the unit this row may not see (mode 1: query token j of n is
+    // n - 1 - j positions before the last one).
+    const int lag = (multi && valid_row) ? p.n_queries - 1 - row / G : 0;
+    if (!split || w == 0) {
       const int n = row / G, g = row % G;
-      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.q) +
-                                                        (static_cast<int64_t>(n) * p.n_q_heads + h * G + g) * kBifD);
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(p.q) +
+          (static_cast<int64_t>(q_tok0 + n) * p.n_q_heads + h * G + g) * kBifD);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const uint4 v = valid_row ? src[c] : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(sm.q[w][c >> 3] + sw128_offset(r, c & 7)) = v;
       }
       fence_proxy_async_smem();
-      mbar_arrive(&sm.q_ready);
     }
+    mbar_arrive(&sm.q_ready);
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    bool ok = w < n_mt;
-    for (int i = 0; ok && i < n_t; ++i) {
+    bool ok = w < n_slots;
+    const int n_w = w >= n_slots ? 0 : (split ? (n_t - w + 1) / 2 : n_t);
+    for (int i = 0; ok && i < n_w; ++i) {
       // S(i) landed; with it, P(i - 1) V(i - 1) is complete (same issuing thread, in order).
       ok = bif_wait(&sm.s_full[w], i & 1, p, abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int64_t nvalid = p.prefix_len - (j0 + i) * kBifKeys;
-      const bool full = nvalid >= kBifKeys;
+      const int tg = split ? 2 * i + w : i;  // the CTA's key tile
+      const int64_t nvalid64 = kv_len - lag - (j0 + tg) * kBifKeys;
+      const int nvalid = static_cast<int>(max(static_cast<int64_t>(-1), min(nvalid64, static_cast<int64_t>(kBifKeys))));
+      // tcgen05.ld is warp-collective: a warp takes the masked path if any of its rows needs it.
+      const bool full = __all_sync(0xffffffffu, nvalid >= kBifKeys);
       // Pass 1: the tile's scaled row max, streamed from TMEM.
-      const float tmax = full ? bif_tile_max(s_col, sc) : bif_tile_max_partial(s_col, sc, static_cast<int>(nvalid));
+      const float tmax = full ? bif_tile_max(s_col, sc) : bif_tile_max_partial(s_col, sc, nvalid);
       const bool need = tmax > m + kBifRescale;
       const float mn = need ? tmax : m;
       // Ping-pong: M tile 1's exponentials of key tile i follow M tile 0's, and M tile 0's of
       // tile i + 1 follow M tile 1's of tile i, so one warpgroup's exponentials overlap the
       // other M tile's products on the tensor pipe.
-      const bool pingpong = kBifPingPong && n_mt == kBifMT;
+      const bool pingpong = kBifPingPong && n_slots == kBifMT;
       if (pingpong && (w == 1 || i >= 1)) {
         ok = bif_wait(&sm.turn[w], (w == 1 ? i : i - 1) & 1, p, abort);
         ok = __all_sync(0xffffffffu, ok);
@@ -616,7 +637,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       }
       // Pass 2: p = 2^(x s - m), summed in fp32, written back as fp16 pairs over the first 64
       // columns of S (P overwrites only columns whose scores were already read).
-      const float rs = full ? bif_tile_exp(s_col, sc, mn) : bif_tile_exp_partial(s_col, sc, mn, static_cast<int>(nvalid));
+      const float rs = full ? bif_tile_exp(s_col, sc, mn) : bif_tile_exp_partial(s_col, sc, mn, nvalid);
       if (pingpong) mbar_arrive(&sm.turn[1 - w]);
       const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
       // O holds tiles 0..i-1 and P(i - 1) V(i - 1) is complete: rescale it when m grew.
@@ -638,14 +659,17 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       mbar_arrive(&sm.p_full[w]);
     }
     // The chunk's statistics of this row.
-    if (w < n_mt) {
-      float* dst =
-          p.part + ((static_cast<int64_t>(chunk) * p.n_kv_heads + h) * p.rows_per_head + row) * kBifPartRow;
-      if (n_t > 0 && ok) {
+    if (w < n_slots) {
+      // Mode 0: [chunk][KV head][row]; mode 1: [sequence, KV head][chunk][slot][row].
+      const int64_t prow =
+          multi ? ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.n_chunks + chunk) * kBifMT + w
+                : static_cast<int64_t>(chunk) * p.n_kv_heads + h;
+      float* dst = p.part + (prow * p.rows_per_head + row) * kBifPartRow;
+      if (n_w > 0 && ok) {
         ok = bif_wait(&sm.o_done[w], 0, p, abort);
         ok = __all_sync(0xffffffffu, ok);
       }
-      if (n_t > 0 && ok) {
+      if (n_w > 0 && ok) {
         tc_fence_after();
 #pragma unroll
         for (int q4 = 0; q4 < kBifD / 32; ++q4) {
@@ -681,6 +705,56 @@ __global__ void __launch_bounds__(kBifThreads, 1)
 // ---------------------------------------------------------------------------------------------
 // Merge: the prefix chunks' statistics with the suffix result, per (sample, query head)
 // ---------------------------------------------------------------------------------------------
+
+// Mode 1: a unit's 2 * n_chunks partials, merged online per output row (b, j, hq); one thread
+// per 4 columns.
+__global__ void __launch_bounds__(128) merge_chunks_kernel(const float* __restrict__ part, int n_chunks,
+                                                           int n_kv_heads, int rows_per_head, int n_queries,
+                                                           float* __restrict__ out, float* __restrict__ lse,
+                                                           int batch, int n_q_heads, const int* __restrict__ err) {
+  constexpr int Q = kBifD / 4;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(batch) * n_queries * n_q_heads * Q;
+  if (i >= total) return;
+  const int d4 = static_cast<int>(i % Q) * 4;
+  const int64_t rq = i / Q;  // (b * n + j) * Hq + hq
+  const int hq = static_cast<int>(rq % n_q_heads);
+  const int64_t bj = rq / n_q_heads;
+  const int j = static_cast<int>(bj % n_queries), b = static_cast<int>(bj / n_queries);
+  const int G = n_q_heads / n_kv_heads;
+  const int h = hq / G, row = j * G + hq % G;
+  const int n_parts = n_chunks * kBifMT;
+  const float* base = part + ((static_cast<int64_t>(b) * n_kv_heads + h) * n_parts * rows_per_head + row) * kBifPartRow;
+  const int64_t stride = static_cast<int64_t>(rows_per_head) * kBifPartRow;
+  float M = -INFINITY, L = 0.f;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+  for (int c = 0; c < n_parts; ++c) {
+    const float* pc = base + c * stride;
+    const float2 ml = *reinterpret_cast<const float2*>(pc);
+    const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
+    if (ml.x == -INFINITY) continue;  // a chunk or slot without keys for this row
+    const float Mn = fmaxf(M, ml.x);
+    const float a = (M == -INFINITY) ? 0.f : ex2(M - Mn);
+    const float bw = ex2(ml.x - Mn);
+    L = L * a + ml.y * bw;
+    O = make_float4(O.x * a + o.x * bw, O.y * a + o.y * bw, O.z * a + o.z * bw, O.w * a + o.w * bw);
+    M = Mn;
+  }
+  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lv = -INFINITY;
+  if (L > 0.f) {
+    ov = make_float4(O.x / L, O.y / L, O.z / L, O.w / L);
+    lv = (M + log2f(L)) * 0.693147180559945309f;
+  }
+  if (*reinterpret_cast<const volatile int*>(err) != 0) {
+    const float nan = __int_as_float(0x7fc00000);
+    ov = make_float4(nan, nan, nan, nan);
+    lv = nan;
+  }
+  *reinterpret_cast<float4*>(out + rq * kBifD + d4) = ov;
+  if (d4 == 0) lse[rq] = lv;
+}
 
 // Suffix part given normalised (out_s, lse_s); it enters as m = lse_s log2(e), l = 1, o = out_s.
 // One thread per 4 columns of an output row.  One online pass over the chunks (the running

@@ -16,6 +16,7 @@ constexpr int kBifD = 128;          // head_dim
 constexpr int kBifThreads = 384;    // 12 warps
 constexpr int kErrBifWait = 4;
 constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
+constexpr int kBifMaxSeq = 128;         // sequences per launch of the several-query-tokens form
 
 struct BifParams {
   const void* q;          // [N][Hq][D] bf16
@@ -29,6 +30,16 @@ struct BifParams {
   int64_t prefix_len;
   float scale_log2;
   int64_t wait_limit_ns;
+  // mode 0: shared prefix; grid (row-tile pairs, chunks, KV heads); rows are the samples'
+  //   query heads of KV head h, each CTA's two M tiles consume every key tile of its chunk.
+  // mode 1: several query tokens per sequence; grid (chunks, KV heads, sequences); a unit's
+  //   rows_per_head = G * n_queries rows (token j, head g at row j * G + g, at most 128) see
+  //   sequence b's keys of KV head h; the CTA's two softmax slots hold the same rows and take
+  //   alternate key tiles; row j * G + g sees the first S_b - n_queries + j + 1 keys.
+  int mode;
+  int n_queries;
+  int64_t kv_row0[kBifMaxSeq];  // mode 1: tensor-map row of key 0 of sequence b, KV head 0
+  int64_t kv_len[kBifMaxSeq];   // mode 1: S_b
 };
 
 // Dynamic shared memory of bif_prefix_kernel (the tile ring plus 1 KB for 1024-byte alignment).
@@ -40,6 +51,10 @@ cudaError_t bif_prefix_set_smem_limit();
 // Prefix pass: grid (M-tile pairs, prefix chunks, KV heads), one CTA per SM.
 cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensorMap& vmap, const BifParams& p,
                               cudaStream_t st);
+
+// Mode 1: merge of a unit's 2 * n_chunks partials into out [B][n][Hq][D] and lse [B][n][Hq].
+cudaError_t launch_merge_chunks(const float* part, int n_chunks, int n_kv_heads, int rows_per_head, int n_queries,
+                                float* out, float* lse, int batch, int n_q_heads, const int* err, cudaStream_t st);
 
 // Merge of the prefix chunks' statistics with the suffix result, per (sample, query head).
 cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,

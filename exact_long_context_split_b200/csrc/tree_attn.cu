@@ -331,6 +331,20 @@ struct MultiPass {
   Plan plan;
 };
 
+// Either split-KV passes, or the tensor-core form: per launch group of at most kBifMaxSeq
+// sequences one bif_prefix_kernel launch in mode 1 (grid chunks x Hkv x sequences) and one
+// merge of each unit's 2 * chunks partials.
+struct MultiPlan {
+  bool tc = false;
+  std::vector<MultiPass> passes;
+  std::vector<int> chunks;  // tensor-core form: chunks per unit of each launch group
+  int rows = 0;
+  size_t body = 0;  // workspace bytes after the header
+};
+
+ta_status bif_tc_setup(int* sms);
+ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows);
+
 ta_status multi_validate(const DecodeArgs& a, int n_queries, const ta_options* opts, bool check_pointers,
                          KernelInfo* ki) {
   if (n_queries < 1) return TA_ERR_INVALID_ARG;
@@ -341,12 +355,40 @@ ta_status multi_validate(const DecodeArgs& a, int n_queries, const ta_options* o
   return TA_OK;
 }
 
-ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts, std::vector<MultiPass>* passes,
-                     size_t* body_max) {
+ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts, MultiPlan* mp_out) {
   const int G = a.Hq / a.Hkv;
+  MultiPlan& P = *mp_out;
+  P = MultiPlan();
+  // Tensor-core form: bf16, head_dim 128, 8..128 rows per unit, cache rows addressable by the
+  // tensor map's 32-bit coordinates.
+  int64_t cache_rows = 0;
+  for (int b = 0; b < a.batch; ++b) cache_rows += a.seqlens[b] * a.Hkv;
+  const int rows = G * n_queries;
+  const bool tc_ok = a.dt == TA_BF16 && a.D == kBifD && rows <= kBifRows && cache_rows < (int64_t(1) << 31) &&
+                     a.kv_offsets == nullptr;
+  const int path = opts ? opts->prefix_path : 0;
+  if (path == 1 && !tc_ok) return TA_ERR_UNSUPPORTED;
+  if (path == 1 || (path == 0 && tc_ok && rows >= 8)) {
+    P.tc = true;
+    P.rows = rows;
+    int sms = 1;
+    if (a.batch > 0) {
+      const ta_status s = bif_tc_setup(&sms);
+      if (s != TA_OK) return s;
+    }
+    size_t part = 0;
+    for (int b0 = 0; b0 < a.batch; b0 += kBifMaxSeq) {
+      const int nb = std::min(kBifMaxSeq, a.batch - b0);
+      int64_t max_tiles = 1;
+      for (int i = 0; i < nb; ++i) max_tiles = std::max<int64_t>(max_tiles, (a.seqlens[b0 + i] + kBifKeys - 1) / kBifKeys);
+      const int64_t c = std::max<int64_t>(1, std::min<int64_t>(sms / (static_cast<int64_t>(nb) * a.Hkv), max_tiles));
+      P.chunks.push_back(static_cast<int>(c));
+      part = std::max(part, sizeof(float) * static_cast<size_t>(nb) * a.Hkv * c * kBifMT * rows * kBifPartRow);
+    }
+    P.body = part;
+    return TA_OK;
+  }
   const bool short_tiles = use_short_tiles(a.seqlens, a.batch, opts);
-  passes->clear();
-  *body_max = 0;
   for (int j0 = 0; j0 < n_queries;) {
     int nq = 1;
     while (2 * nq <= n_queries - j0 && G * 2 * nq <= 8) nq *= 2;
@@ -362,22 +404,63 @@ ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts,
     const ta_status s = build_plan(a.seqlens, a.kv_offsets, a.batch, a.Hkv, G * nq, a.D, mp.ki.tile, slots, opts,
                                    &mp.plan);
     if (s != TA_OK) return s;
-    *body_max = std::max(*body_max, mp.plan.body_bytes);
-    passes->push_back(mp);
+    P.body = std::max(P.body, mp.plan.body_bytes);
+    P.passes.push_back(mp);
     j0 += nq;
   }
   return TA_OK;
 }
 
-ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, const std::vector<MultiPass>& passes,
-                    void* ws, size_t ws_bytes, size_t body_max, cudaStream_t st) {
-  if (!ws || !aligned(ws, kAlign) || ws_bytes < kHeaderBytes + body_max) return TA_ERR_WORKSPACE;
+ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, const MultiPlan& P, void* ws,
+                    size_t ws_bytes, cudaStream_t st) {
+  if (!ws || !aligned(ws, kAlign) || ws_bytes < kHeaderBytes + P.body) return TA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
-  for (const MultiPass& mp : passes) {
-    const ta_status s = launch_plan(mp.plan, mp.ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt,
-                                    opts, base + kHeaderBytes, reinterpret_cast<int*>(base), st, n_queries,
-                                    mp.q_first);
-    if (s != TA_OK) return s;
+  int* err = reinterpret_cast<int*>(base);
+  if (!P.tc) {
+    for (const MultiPass& mp : P.passes) {
+      const ta_status s = launch_plan(mp.plan, mp.ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt,
+                                      opts, base + kHeaderBytes, err, st, n_queries, mp.q_first);
+      if (s != TA_OK) return s;
+    }
+    return TA_OK;
+  }
+  int64_t cache_rows = 0;
+  for (int b = 0; b < a.batch; ++b) cache_rows += a.seqlens[b] * a.Hkv;
+  CUtensorMap kmap, vmap;
+  ta_status s = encode_cache_map(&kmap, a.k, cache_rows);
+  if (s != TA_OK) return s;
+  s = encode_cache_map(&vmap, a.v, cache_rows);
+  if (s != TA_OK) return s;
+  float* part = reinterpret_cast<float*>(base + kHeaderBytes);
+  int64_t row0 = 0;  // tensor-map row of the group's first sequence
+  for (int b0 = 0; b0 < a.batch; b0 += kBifMaxSeq) {
+    const int nb = std::min(kBifMaxSeq, a.batch - b0);
+    BifParams bp;
+    std::memset(&bp, 0, sizeof(bp));
+    const size_t qrow0 = static_cast<size_t>(b0) * n_queries * a.Hq;
+    bp.q = static_cast<const uint8_t*>(a.q) + qrow0 * a.D * 2;
+    bp.part = part;
+    bp.err = err;
+    bp.n_samples = nb;
+    bp.n_q_heads = a.Hq;
+    bp.n_kv_heads = a.Hkv;
+    bp.rows_per_head = P.rows;
+    for (int i = 0; i < nb; ++i) {
+      bp.kv_row0[i] = row0;
+      bp.kv_len[i] = a.seqlens[b0 + i];
+      row0 += a.seqlens[b0 + i] * a.Hkv;
+    }
+    bp.n_chunks = P.chunks[b0 / kBifMaxSeq];
+    bp.prefix_len = 0;
+    bp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
+    bp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+    bp.mode = 1;
+    bp.n_queries = n_queries;
+    cudaError_t e = launch_bif_prefix(dim3(bp.n_chunks, a.Hkv, nb), kmap, vmap, bp, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = launch_merge_chunks(part, bp.n_chunks, a.Hkv, P.rows, n_queries, a.out + qrow0 * a.D, a.lse + qrow0, nb,
+                            a.Hq, err, st);
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return TA_OK;
 }
@@ -462,6 +545,12 @@ bool encode_kv_map(CUtensorMap* map, const void* base, int64_t rows) {
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The whole packed cache as one [rows][128] bf16 matrix for the tensor-core passes.
+ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows) {
+  if (rows <= 0) rows = 1;  // no key is read; the map only has to be valid
+  return encode_kv_map(map, base, rows) ? TA_OK : TA_ERR_UNSUPPORTED;
 }
 
 ta_status bif_tc_setup(int* sms) {
@@ -756,11 +845,10 @@ ta_status tree_attn_multi_workspace_size(const int64_t* seqlens, int32_t batch, 
   KernelInfo ki;
   ta_status s = multi_validate(a, n_queries, opts, false, &ki);
   if (s != TA_OK) return s;
-  std::vector<MultiPass> passes;
-  size_t body = 0;
-  s = multi_plan(a, n_queries, opts, &passes, &body);
+  MultiPlan plan;
+  s = multi_plan(a, n_queries, opts, &plan);
   if (s != TA_OK) return s;
-  *bytes = kHeaderBytes + body;
+  *bytes = kHeaderBytes + plan.body;
   return TA_OK;
 }
 
@@ -774,23 +862,21 @@ ta_status tree_attn_decode_multi_ex(ta_dtype dtype, const void* q, const void* k
   KernelInfo ki;
   ta_status s = multi_validate(a, n_queries, opts, true, &ki);
   if (s != TA_OK || batch == 0) return s;
-  std::vector<MultiPass> passes;
-  size_t body = 0;
-  s = multi_plan(a, n_queries, opts, &passes, &body);
+  MultiPlan plan;
+  s = multi_plan(a, n_queries, opts, &plan);
   if (s != TA_OK) return s;
-  return multi_run(a, n_queries, opts, passes, workspace, workspace_bytes, body, static_cast<cudaStream_t>(stream));
+  return multi_run(a, n_queries, opts, plan, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 namespace {
 struct MultiCtx {
   DecodeArgs a;
   int n_queries;
-  const std::vector<MultiPass>* passes;
-  size_t body;
+  const MultiPlan* plan;
 };
 ta_status multi_alloc_run(void* ws, size_t bytes, void* ctx, cudaStream_t st) {
   MultiCtx* c = static_cast<MultiCtx*>(ctx);
-  return multi_run(c->a, c->n_queries, nullptr, *c->passes, ws, bytes, c->body, st);
+  return multi_run(c->a, c->n_queries, nullptr, *c->plan, ws, bytes, st);
 }
 }  // namespace
 
@@ -802,12 +888,11 @@ ta_status tree_attn_decode_multi(const void* q, const void* k_cache, const void*
   KernelInfo ki;
   ta_status s = multi_validate(a, n_queries, nullptr, true, &ki);
   if (s != TA_OK || batch == 0) return s;
-  std::vector<MultiPass> passes;
-  size_t body = 0;
-  s = multi_plan(a, n_queries, nullptr, &passes, &body);
+  MultiPlan plan;
+  s = multi_plan(a, n_queries, nullptr, &plan);
   if (s != TA_OK) return s;
-  MultiCtx ctx{a, n_queries, &passes, body};
-  return with_temp_workspace(kHeaderBytes + body, static_cast<cudaStream_t>(stream), &multi_alloc_run, &ctx);
+  MultiCtx ctx{a, n_queries, &plan};
+  return with_temp_workspace(kHeaderBytes + plan.body, static_cast<cudaStream_t>(stream), &multi_alloc_run, &ctx);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -79,9 +79,12 @@ typedef struct {
                               kernel records TA_ERR_TIMEOUT in the workspace and returns */
   int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
                               consumers' wait runs out (no fault: the data simply never arrives) */
-  int32_t prefix_path;     /* bifurcated calls only.  0: automatic (tensor-core prefix pass when
-                              head_dim is 128 and the prefix is not empty); 1: tensor-core pass
-                              (TA_ERR_UNSUPPORTED if not possible); 2: split-KV pass per sample */
+  int32_t prefix_path;     /* bifurcated and multi-query calls.  Bifurcated: 0 automatic (tensor-
+                              core prefix pass when head_dim is 128 and the prefix is not empty);
+                              1 tensor-core pass (TA_ERR_UNSUPPORTED if not possible); 2 split-KV
+                              pass per sample.  Multi-query: 0 automatic (tensor cores when bf16,
+                              head_dim 128 and 8 <= G * n <= 128); 1 tensor cores; 2 split-KV
+                              passes */
   int32_t split_tiles;     /* split-KV tile configuration.  0: automatic (short tiles when the mean
                               sequence is under 1024 tokens); 1: long tiles; 2: short tiles */
   int32_t reserved[3];     /* must be 0 */
@@ -146,9 +149,12 @@ ta_status tree_attn_decode_ex(ta_dtype dtype, const void* q, const void* k_cache
  *   q    [B][n][Hq][D]  bf16 (or f32 with TA_F32)
  *   k, v packed per sequence as for tree_attn_decode; every S_b >= n, else TA_ERR_INVALID_ARG
  *   out  [B][n][Hq][D]  f32;  lse [B][n][Hq] f32
- * One pass over the cache serves G * n' rows per KV head (n' consecutive query tokens, a power
- * of two, G * n' <= 8, G = n_q_heads / n_kv_heads); larger n takes several passes, run in turn
- * on `stream` with one workspace.  Other rules as tree_attn_decode / tree_attn_decode_ex.
+ * Two forms (ta_options.prefix_path).  Tensor cores (bf16, head_dim 128, G * n <= 128 with
+ * G = n_q_heads / n_kv_heads): the G * n rows of a (sequence, KV head) form one matrix that
+ * reads the cache once, S = Q K^T and O = P V on tcgen05, chunked over the SMs and merged
+ * exactly.  Split-KV: one pass over the cache serves G * n' rows per KV head (n' consecutive
+ * query tokens, a power of two, G * n' <= 8); larger n takes several passes, run in turn on
+ * `stream` with one workspace.  Other rules as tree_attn_decode / tree_attn_decode_ex.
  */
 ta_status tree_attn_multi_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_queries,
                                          int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, ta_dtype dtype,

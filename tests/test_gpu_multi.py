@@ -61,27 +61,69 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("tiles", [1, 2])
+def tc_eligible(n, Hq, Hkv, D, dtype):
+    return dtype == "bf16" and D == 128 and (Hq // Hkv) * n <= 128
+
+
+# path: 0 automatic (tensor cores when bf16, D = 128 and 8 <= G n <= 128), 1 tensor-core form,
+# 2 split-KV passes (with long or short tiles).
+@pytest.mark.parametrize("path,tiles", [(0, 0), (1, 0), (2, 1), (2, 2)])
 @pytest.mark.parametrize("case", CASES, ids=[f"n{c[1]}_G{c[2] // c[3]}_D{c[4]}_{c[5]}" for c in CASES])
-def test_multi_query_against_oracle(case, tiles):
+def test_multi_query_against_oracle(case, path, tiles):
     import exact_long_context_split_b200 as ta
 
     seqlens, n, Hq, Hkv, D, dtype = case
     sp = spec(seqlens, n, Hq, Hkv, D, dtype=dtype, seed=40 + n + D)
     inp = synth.make_decode_inputs(sp)
-    out, lse = multi_gpu(inp, sp, ta.make_options(split_tiles=tiles))
+    opts = ta.make_options(split_tiles=tiles, prefix_path=path)
+    if path == 1 and not tc_eligible(n, Hq, Hkv, D, dtype):
+        with pytest.raises(ta.TreeAttnError) as e:
+            multi_gpu(inp, sp, opts)
+        assert e.value.status == ta.TA_ERR_UNSUPPORTED
+        return
+    out, lse = multi_gpu(inp, sp, opts)
     check(out, lse, inp, sp)
+
+
+# Tensor-core form: shorter than one 128-key tile, on and next to tile boundaries, G n = 128
+# rows, and more than 128 sequences (two launch groups with their own chunk counts).
+TC_CASES = [
+    ([5, 128, 129, 256, 257], 4, 16, 4, 1),
+    ([3000, 16], 16, 64, 8, 3),
+    ([70] * 130 + [5000], 2, 8, 2, 5),
+    ([1000, 40000], 3, 32, 8, 7),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=["tile_edges", "rows128", "two_groups", "long"])
+def test_tensor_core_multi_query(case):
+    import exact_long_context_split_b200 as ta
+
+    seqlens, n, Hq, Hkv, seed = case
+    sp = spec(seqlens, n, Hq, Hkv, 128, seed=seed)
+    inp = synth.make_decode_inputs(sp)
+    opts = ta.make_options(prefix_path=1)
+    out, lse = multi_gpu(inp, sp, opts)
+    r = np.random.default_rng(seed)
+    rows = None
+    if sp.batch * n * Hq > 400:
+        rows = sorted({(int(r.integers(sp.batch)), int(r.integers(n)), int(r.integers(Hq))) for _ in range(150)} |
+                      {(sp.batch - 1, j, h) for j in range(n) for h in (0, Hq - 1)})
+    check(out, lse, inp, sp, rows=rows)
+    out2, lse2 = multi_gpu(inp, sp, opts)
+    assert np.array_equal(out.view(np.uint32), out2.view(np.uint32)), "not bit-identical across runs"
+    assert np.array_equal(lse.view(np.uint32), lse2.view(np.uint32))
 
 
 @pytest.mark.parametrize("num_ctas", [1, 3, 148, 100000])
 def test_masked_tail_alone_in_a_cta(num_ctas):
-    """One tile per CTA: the CTA holding a sequence's last tile (2 tokens) sees no key for the
-    query tokens that precede them, and sends an empty partial to the merge."""
+    """Split-KV passes with one tile per CTA: the CTA holding a sequence's last tile (2 tokens)
+    sees no key for the query tokens that precede them, and sends an empty partial."""
     import exact_long_context_split_b200 as ta
 
     sp = spec([130, 66], 4, 8, 2, 128, seed=77)
     inp = synth.make_decode_inputs(sp)
-    opts = ta.make_options(num_ctas=num_ctas, split_tiles=2)
+    opts = ta.make_options(num_ctas=num_ctas, split_tiles=2, prefix_path=2)
     out, lse = multi_gpu(inp, sp, opts)
     check(out, lse, inp, sp)
     out2, lse2 = multi_gpu(inp, sp, opts)
@@ -92,9 +134,11 @@ def test_one_query_equals_decode():
     """n = 1 runs the decode kernels with the same plan: bit-identical to tree_attn_decode_ex."""
     from gpu_util import decode_gpu
 
+    import exact_long_context_split_b200 as ta
+
     sp1 = spec([17, 2000, 40000], 1, 32, 8, 128, seed=5)
     inp = synth.make_decode_inputs(sp1)
-    out, lse = multi_gpu(inp, sp1)
+    out, lse = multi_gpu(inp, sp1, ta.make_options(prefix_path=2))
     sp = synth.DecodeSpec("plain", [17, 2000, 40000], 32, 8, 128, seed=5)
     ref_out, ref_lse = decode_gpu(synth.make_decode_inputs(sp), sp)
     assert np.array_equal(out[:, 0].view(np.uint32), ref_out.view(np.uint32))
