@@ -15,10 +15,12 @@ from .attention import (  # noqa: F401
     decode_attention,
     energy,
     finalize,
+    gather_paged_sequence,
     merge,
     merge_tree,
     multi_query_attention,
     online_softmax,
+    paged_decode_attention,
     sequence_block,
     split_attention,
     to_f64,

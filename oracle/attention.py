@@ -46,6 +46,11 @@ design notes):
    token j (0-based) sits at position S - n + j and attends to every key at or before it,
    i.e. to the first S - n + j + 1 keys (all preceding context, causal among the n new
    tokens).  n = 1 is ordinary decode.
+8. Paged cache ([AttnAccel] part 3, "PagedAttention (vLLM)"): the cache is cut into blocks of
+   a fixed number of tokens and a table maps each sequence's logical blocks to physical ones
+   (which sequences may share).  Layout read here: physical block p holds, for each KV head
+   h, page_size consecutive token rows [p][h][0..page_size)[D]; logical block i of sequence b
+   (its tokens i * page_size ...) is physical block table[b][i].
 """
 from __future__ import annotations
 
@@ -334,3 +339,28 @@ def multi_query_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_queries
             out[b, j, h], lse[b, j, h] = attention_one_bf16_cache(qf[b, j, h], Kb[g][:visible], Vb[g][:visible],
                                                                   scale, dtype)
     return out, lse
+
+
+def gather_paged_sequence(pages, block_row, seqlen: int, n_kv_heads: int, page_size: int, head_dim: int):
+    """Sequence b's [Hkv][S][D] block read through its row of the block table (reading 8):
+    token t of KV head h is row t % page_size of head h in physical block block_row[t // page_size]."""
+    S, Hkv, ps, D = int(seqlen), n_kv_heads, page_size, head_dim
+    pages = np.asarray(pages).reshape(-1, Hkv, ps, D)
+    out = np.empty((Hkv, S, D), dtype=pages.dtype)
+    for t in range(S):
+        out[:, t, :] = pages[int(block_row[t // ps]), :, t % ps, :]
+    return out
+
+
+def paged_decode_attention(q, k_pages, v_pages, block_table, seqlens: Sequence[int], page_size: int,
+                           n_q_heads: int, n_kv_heads: int, head_dim: int, scale: float, dtype: str = "bf16",
+                           pairs: Optional[Iterable[Tuple[int, int]]] = None):
+    """Decode attention over a paged cache (reading 8): each sequence's cache is gathered through
+    its block-table row, then attended exactly as decode_attention does.  block_table: [B][*]."""
+    B = len(seqlens)
+    Hkv, D = n_kv_heads, head_dim
+    blocks = [gather_paged_sequence(k_pages, block_table[b], seqlens[b], Hkv, page_size, D) for b in range(B)]
+    kc = np.concatenate([x.reshape(-1) for x in blocks]) if B else np.zeros(0, dtype=np.asarray(k_pages).dtype)
+    blocks = [gather_paged_sequence(v_pages, block_table[b], seqlens[b], Hkv, page_size, D) for b in range(B)]
+    vc = np.concatenate([x.reshape(-1) for x in blocks]) if B else np.zeros(0, dtype=np.asarray(v_pages).dtype)
+    return decode_attention(q, kc, vc, seqlens, n_q_heads, n_kv_heads, head_dim, scale, dtype=dtype, pairs=pairs)

@@ -451,6 +451,55 @@ def pin_multi_query(O):
             _close(lse1[b, 0, h], x.max() + math.log(e.sum()), rtol=1e-13, what="n = 1 lse")
 
 
+def pin_paged_cache(O):
+    """[AttnAccel] part 3 (reading 8): a contiguous cache scattered into pages through a random
+    block table (numpy fancy indexing, page by page, independent of the oracle's token loop)
+    gives back every sequence's cache, and paged decode then equals decode of the contiguous
+    cache; two sequences whose tables share their first blocks see the same prefix rows."""
+    r = _rng(23)
+    D, Hkv, Hq, ps = 4, 2, 4, 4
+    seqlens = [9, 4, 13, 1]
+    blocks_per = [-(-S // ps) for S in seqlens]
+    n_pages = sum(blocks_per) + 3
+    perm = r.permutation(n_pages)
+    table = np.full((len(seqlens), max(blocks_per)), -1, dtype=np.int64)
+    pages_k = r.standard_normal((n_pages, Hkv, ps, D))
+    pages_v = r.standard_normal((n_pages, Hkv, ps, D))
+    caches_k, caches_v = [], []
+    used = 0
+    for b, S in enumerate(seqlens):
+        kb = r.standard_normal((Hkv, S, D))
+        vb = r.standard_normal((Hkv, S, D))
+        caches_k.append(kb)
+        caches_v.append(vb)
+        for i in range(blocks_per[b]):
+            p = int(perm[used])
+            used += 1
+            table[b, i] = p
+            n = min(ps, S - i * ps)
+            pages_k[p, :, :n, :] = kb[:, i * ps:i * ps + n, :]
+            pages_v[p, :, :n, :] = vb[:, i * ps:i * ps + n, :]
+    for b, S in enumerate(seqlens):
+        got = O.gather_paged_sequence(pages_k.reshape(-1), table[b], S, Hkv, ps, D)
+        _close(got, caches_k[b], rtol=0.0, what=f"gathered cache {b}")
+    q = r.standard_normal((len(seqlens), Hq, D))
+    out, lse = O.paged_decode_attention(q, pages_k.reshape(-1), pages_v.reshape(-1), table, seqlens, ps, Hq, Hkv, D,
+                                        0.6, dtype="f64")
+    G = Hq // Hkv
+    for b, S in enumerate(seqlens):
+        for h in range(Hq):
+            x = 0.6 * (caches_k[b][h // G] @ q[b, h])
+            e = np.exp(x - x.max())
+            _close(out[b, h], (e @ caches_v[b][h // G]) / e.sum(), rtol=1e-12, atol=1e-14, what=f"paged {b},{h}")
+            _close(lse[b, h], x.max() + math.log(e.sum()), rtol=1e-13, what=f"paged lse {b},{h}")
+    # shared prefix blocks: sequence 1 reuses sequence 0's first block
+    shared = table.copy()
+    shared[1, 0] = table[0, 0]
+    g0 = O.gather_paged_sequence(pages_v.reshape(-1), shared[0], seqlens[0], Hkv, ps, D)
+    g1 = O.gather_paged_sequence(pages_v.reshape(-1), shared[1], seqlens[1], Hkv, ps, D)
+    _close(g1[:, :ps], g0[:, :ps], rtol=0.0, what="shared block")
+
+
 ALL_PINS = [
     pin_bf16_decoding,
     pin_identical_keys,
@@ -471,4 +520,5 @@ ALL_PINS = [
     pin_bifurcated,
     pin_long_cache_pieces,
     pin_multi_query,
+    pin_paged_cache,
 ]

@@ -36,6 +36,8 @@ MUTANTS = {
                                        "Ks = to_f64(sequence_block(k_suffix, suffix_lens, 0, Hkv, D), dtype)\n        Vs = to_f64(sequence_block(v_suffix, suffix_lens, 0, Hkv, D), dtype)"),
     "multi-query mask one short": ("            visible = S - n + j + 1\n", "            visible = S - n + j\n"),
     "multi-query mask reversed": ("            visible = S - n + j + 1\n", "            visible = S - j\n"),
+    "paged block index off by one": ("pages[int(block_row[t // ps]), :, t % ps, :]", "pages[int(block_row[t // ps + (t >= ps)]), :, t % ps, :]"),
+    "paged rows ignore the head": ("pages[int(block_row[t // ps]), :, t % ps, :]", "pages[int(block_row[t // ps]), :1, t % ps, :]"),
     "pieces skip last rows": ("        acc += e[r0:r1] @ to_f64(Vbits[r0:r1], dtype)", "        acc += e[r0:r1 - (r1 == S)] @ to_f64(Vbits[r0:r1 - (r1 == S)], dtype)"),
 }
 
