@@ -195,7 +195,7 @@ def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra
         "config": {
             "workload": spec.name,
             **({"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
-                "query_tokens": spec.n_queries}
+                "query_tokens": spec.n_queries, **({"page_size": spec.page_size} if spec.page_size else {})}
                if isinstance(spec, synth.DecodeSpec) else
                {"samples": spec.n_samples, "prefix_len": spec.prefix_len,
                 "suffix_len": int(max(spec.suffix_lens)) if spec.suffix_lens else 0}),
@@ -347,6 +347,37 @@ class MultiRun(DecodeRun):
                                           self.lse, None, self.ws, stream=stream)
 
 
+class PagedRun(DecodeRun):
+    """A paged cache: the contiguous cache laid out in page_size-token blocks at seeded random
+    places (built once on the device); each step reads it through the block table."""
+
+    def __init__(self, spec, torch, ta):
+        super().__init__(spec, torch, ta)
+        Hkv, D, ps = spec.n_kv_heads, spec.head_dim, spec.page_size
+        table, self.num_pages = synth.page_table(spec.seed, spec.seqlens, ps)
+        self.table = torch.from_numpy(table).cuda()
+        self.stride = table.shape[1]
+        for name in ("k", "v"):
+            pages = torch.zeros(self.num_pages, Hkv, ps, D, dtype=torch.bfloat16, device="cuda")
+            off = 0
+            for b, S in enumerate(self.seqlens):
+                nb = -(-S // ps)
+                blk = torch.zeros(Hkv, nb * ps, D, dtype=torch.bfloat16, device="cuda")
+                blk[:, :S] = self.dev[name][off:off + Hkv * S * D].view(Hkv, S, D)
+                off += Hkv * S * D
+                pages[self.table[b, :nb].long()] = blk.view(Hkv, nb, ps, D).permute(1, 0, 2, 3)
+            self.dev[name] = pages.view(-1)
+            self.host[name] = pages.view(-1).cpu().pin_memory()  # the end-to-end leg uploads pages
+        self.kernel += " (paged, %d-token blocks)" % ps
+
+    def step(self, stream):
+        sp = self.spec
+        self.ta.tree_attn_decode_paged_ex("bf16", self.dev["q"], self.dev["k"], self.dev["v"], self.num_pages,
+                                          sp.page_size, self.table, self.stride, self.seqlens, sp.n_q_heads,
+                                          sp.n_kv_heads, sp.head_dim, sp.scale, self.out, self.lse, None, self.ws,
+                                          stream=stream)
+
+
 class BifurcatedRun:
     """Shared-prefix workload: one call = prefix pass, suffix pass and the exact merge."""
 
@@ -396,6 +427,8 @@ def run_gpu(args, spec) -> None:
         run = BifurcatedRun(spec, torch, ta)
     elif spec.n_queries > 1:
         run = MultiRun(spec, torch, ta)
+    elif spec.page_size > 0:
+        run = PagedRun(spec, torch, ta)
     else:
         run = DecodeRun(spec, torch, ta)
     stream = torch.cuda.current_stream()
@@ -496,7 +529,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     workloads = {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs(),
-                 **synth.multi_query_configs()}
+                 **synth.multi_query_configs(), **synth.paged_configs()}
     ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

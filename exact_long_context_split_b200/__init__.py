@@ -16,6 +16,7 @@ from ._build import LIB, build  # noqa: F401
 
 TA_OK, TA_ERR_INVALID_ARG, TA_ERR_UNSUPPORTED, TA_ERR_WORKSPACE, TA_ERR_CUDA, TA_ERR_TIMEOUT = range(6)
 TA_ERR_SCRATCH_LIMIT = 6
+TA_ERR_BAD_PAGE = 7
 TA_BF16, TA_F32 = 0, 1
 _DTYPES = {"bf16": TA_BF16, "f32": TA_F32}
 
@@ -35,6 +36,8 @@ EXPORTED = [
     "tree_attn_multi_workspace_size",
     "tree_attn_decode_multi_ex",
     "tree_attn_decode_multi",
+    "tree_attn_decode_paged_ex",
+    "tree_attn_decode_paged",
 ]
 
 
@@ -111,6 +114,12 @@ def lib() -> ctypes.CDLL:
                 ctypes.c_int,
             ),
             "tree_attn_decode_multi": ([vp, vp, vp, pi64, i32, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
+            "tree_attn_decode_paged_ex": (
+                [ctypes.c_int, vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, popt, vp, sz, vp],
+                ctypes.c_int,
+            ),
+            "tree_attn_decode_paged": (
+                [vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(L, name)
@@ -282,3 +291,26 @@ def tree_attn_decode_multi(q, k_cache, v_cache, seqlens, n_queries, n_q_heads, n
     _check(lib().tree_attn_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), arr, n, n_queries, n_q_heads,
                                         n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
            "tree_attn_decode_multi")
+
+
+def tree_attn_decode_paged_ex(dtype, q, k_pages, v_pages, num_pages, page_size, block_table, block_table_stride,
+                              seqlens, n_q_heads, n_kv_heads, head_dim, scale, out, lse, opts, workspace,
+                              workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """Decode over a paged cache: pages [num_pages][Hkv][page_size][D], a device int32 block table."""
+    arr, n = _lens(seqlens)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().tree_attn_decode_paged_ex(_DTYPES[dtype], _ptr(q), _ptr(k_pages), _ptr(v_pages), num_pages,
+                                           page_size, _ptr(block_table), block_table_stride, arr, n, n_q_heads,
+                                           n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse), _opts(opts),
+                                           _ptr(workspace), workspace_bytes, _stream(stream, q, out)),
+           "tree_attn_decode_paged_ex")
+
+
+def tree_attn_decode_paged(q, k_pages, v_pages, num_pages, page_size, block_table, block_table_stride, seqlens,
+                           n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream=None) -> None:
+    arr, n = _lens(seqlens)
+    _check(lib().tree_attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), num_pages, page_size,
+                                        _ptr(block_table), block_table_stride, arr, n, n_q_heads, n_kv_heads,
+                                        head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
+           "tree_attn_decode_paged")

@@ -733,10 +733,11 @@ __global__ void __launch_bounds__(128) merge_chunks_kernel(const float* __restri
     const float* pc = base + c * stride;
     const float2 ml = *reinterpret_cast<const float2*>(pc);
     const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
-    if (ml.x == -INFINITY) continue;  // a chunk or slot without keys for this row
+    // No branch: a chunk or slot without keys for this row (m = -inf) gets weight 0, so the
+    // loads of the whole unrolled group issue together.
     const float Mn = fmaxf(M, ml.x);
     const float a = (M == -INFINITY) ? 0.f : ex2(M - Mn);
-    const float bw = ex2(ml.x - Mn);
+    const float bw = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - Mn);
     L = L * a + ml.y * bw;
     O = make_float4(O.x * a + o.x * bw, O.y * a + o.y * bw, O.z * a + o.z * bw, O.w * a + o.w * bw);
     M = Mn;
@@ -785,10 +786,11 @@ __global__ void __launch_bounds__(128) merge_prefix_suffix_kernel(
     const float* pc = base + c * stride;
     const float2 ml = *reinterpret_cast<const float2*>(pc);
     const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
-    if (ml.x == -INFINITY) continue;  // empty chunk
+    // No branch: an empty chunk (m = -inf) gets weight 0, so the loads of the whole unrolled
+    // group issue together.
     const float Mn = fmaxf(M, ml.x);
     const float a = (M == -INFINITY) ? 0.f : ex2(M - Mn);
-    const float b = ex2(ml.x - Mn);
+    const float b = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - Mn);
     L = L * a + ml.y * b;
     O = make_float4(O.x * a + o.x * b, O.y * a + o.y * b, O.z * a + o.z * b, O.w * a + o.w * b);
     M = Mn;

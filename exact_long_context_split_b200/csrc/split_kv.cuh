@@ -38,6 +38,7 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kErrConsumerWait = 1;
 constexpr int kErrProducerWait = 2;
 constexpr int kErrDrainWait = 3;
+constexpr int kErrBadPage = 8;  // a block-table entry outside [0, num_pages): nothing was read for it
 
 struct SplitParams {
   const void* q;   // [B][Hq][D], this launch's first sequence
@@ -64,6 +65,13 @@ struct SplitParams {
   int32_t n_queries;
   int32_t q_first;
   int32_t log2_heads;
+  // Paged cache (block_table != nullptr): k and v are [num_pages][Hkv][page_size][D]; sequence
+  // b's logical block i (tokens i * page_size ...) is physical block block_table[b * bt_stride + i].
+  // kv_off is unused then.
+  const int32_t* block_table;  // this launch's first sequence's row
+  int64_t bt_stride;
+  int64_t num_pages;
+  int32_t log2_page;
   int64_t kv_off[kMaxSeqPerLaunch];
   int64_t seq_len[kMaxSeqPerLaunch];
   int64_t tile_off[kMaxSeqPerLaunch + 1];  // first tile of sequence b on the line
@@ -372,7 +380,9 @@ __device__ __forceinline__ void write_final(const SplitParams& p, int b, int h, 
 // The kernel
 // ---------------------------------------------------------------------------------------------
 
-template <typename T, int D, int G, class V>
+// PAGED: the cache is read through p.block_table (a separate instance, so the contiguous
+// kernels carry none of the paged producer's code).
+template <typename T, int D, int G, class V, bool PAGED = false>
 __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
     split_kv_decode_kernel(const __grid_constant__ SplitParams p) {
   using C = SplitCfg<T, D, G, V>;
@@ -404,60 +414,162 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
 
   if (warp == C::NCW) {
     // ------------------------------- producer -------------------------------
-    if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      TileWalk w;
-      w.init(p, t_lo);
-      int fills[C::NSTAGE];
+    const uint64_t pol = l2_policy_evict_first();
+    TileWalk w;
+    w.init(p, t_lo);
+    int fills[C::NSTAGE];
 #pragma unroll
-      for (int s = 0; s < C::NSTAGE; ++s) fills[s] = 0;
-      for (int i = 0; i < n_my; ++i) {
-        const int s = i % C::NSTAGE;
-        if (i >= C::NSTAGE) {
-          if (!wait_phase(&sm.empty[s], ((i / C::NSTAGE) - 1) & 1, p.wait_limit_ns, abort_flag)) {
-            if (!*abort_flag) atomicCAS(p.err, 0, kErrProducerWait);
-            *abort_flag = 1;
+    for (int st = 0; st < C::NSTAGE; ++st) fills[st] = 0;
+    if constexpr (!PAGED) {
+      // Contiguous cache: lane 0 alone waits for each stage and issues at once (the ring is
+      // only NSTAGE deep, so any delay between "stage free" and "copies issued" is on the
+      // critical path).
+      if (lane == 0) {
+        for (int i = 0; i < n_my; ++i) {
+          const int s = i % C::NSTAGE;
+          if (i >= C::NSTAGE) {
+            if (!wait_phase(&sm.empty[s], ((i / C::NSTAGE) - 1) & 1, p.wait_limit_ns, abort_flag)) {
+              if (!*abort_flag) atomicCAS(p.err, 0, kErrProducerWait);
+              *abort_flag = 1;
+            }
+          }
+          if (*abort_flag) break;
+          const int64_t len = p.seq_len[w.b];
+          const int64_t t0 = w.j * C::TILE;
+          const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - t0));
+          if (!(cta == 0 && i == p.debug_skip_tile)) {
+            const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
+            constexpr uint32_t q_bytes = G * D * C::ELEM;
+            const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
+            uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
+            mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
+            if (with_q) {
+              // One copy per query token of the launch: its `heads` query heads are contiguous.
+              const int heads = 1 << p.log2_heads;
+              const uint32_t qb = static_cast<uint32_t>(heads) * D * C::ELEM;
+              for (int jl = 0; jl < (G >> p.log2_heads); ++jl) {
+                const uint8_t* qsrc =
+                    reinterpret_cast<const uint8_t*>(p.q) +
+                    ((static_cast<int64_t>(w.b) * p.n_queries + p.q_first + jl) * p.n_q_heads + w.h * heads) * D *
+                        C::ELEM;
+                bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
+              }
+            }
+            if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
+            if (bytes != 0) {
+              const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
+              bulk_load(sm.k[s], reinterpret_cast<const T*>(p.k) + off, bytes, &sm.full[s], pol);
+              bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, vbar, pol);
+            }
+            ++fills[s];
+          }
+          w.next(p);
+        }
+      }
+    } else {
+      uint64_t* const vbar0 = TA_SPLIT_KV_BARRIERS ? sm.full_v : sm.full;
+      // Stage s's expected bytes and the unit's q, which lands with the unit's first tile (one
+      // copy per query token of the launch: its `heads` query heads are contiguous).  Lane 0.
+      auto tile_header = [&](int s, int i, uint32_t bytes) {
+        constexpr uint32_t q_bytes = G * D * C::ELEM;
+        const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
+        mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
+        if (with_q) {
+          const int heads = 1 << p.log2_heads;
+          const uint32_t qb = static_cast<uint32_t>(heads) * D * C::ELEM;
+          for (int jl = 0; jl < (G >> p.log2_heads); ++jl) {
+            const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q) +
+                                  ((static_cast<int64_t>(w.b) * p.n_queries + p.q_first + jl) * p.n_q_heads +
+                                   w.h * heads) * D * C::ELEM;
+            bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
           }
         }
-        if (*abort_flag) break;
+        if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(&vbar0[s], bytes);
+      };
+      auto stage_wait = [&](int s, int i) {  // lane 0: the stage's previous tile was consumed
+        if (i >= C::NSTAGE && !wait_phase(&sm.empty[s], ((i / C::NSTAGE) - 1) & 1, p.wait_limit_ns, abort_flag)) {
+          if (!*abort_flag) atomicCAS(p.err, 0, kErrProducerWait);
+          *abort_flag = 1;
+        }
+      };
+      // Paged cache: one copy per page a tile touches, lane k taking page k (at most 25 pages:
+      // 384-token tiles of 16-token pages).  Each lane loads its block-table entry one tile
+      // ahead; the warp checks a tile's entries against num_pages before anything is expected
+      // on the stage's barrier, so nothing is ever read through a bad entry.
+      auto fetch = [&](const TileWalk& tw, int64_t* page, int* n_pg, bool* bad) {
+        const int64_t len = p.seq_len[tw.b];
+        const int64_t t0 = tw.j * C::TILE;
+        const int64_t nv = min(static_cast<int64_t>(C::TILE), len - t0);
+        *page = 0;
+        *n_pg = 0;
+        *bad = false;
+        if (nv > 0) {
+          const int64_t pg0 = t0 >> p.log2_page;
+          *n_pg = static_cast<int>(((t0 + nv - 1) >> p.log2_page) - pg0 + 1);
+          if (lane < *n_pg) {
+            *page = __ldg(p.block_table + tw.b * p.bt_stride + pg0 + lane);
+            *bad = *page < 0 || *page >= p.num_pages;
+          }
+        }
+      };
+      int64_t page = 0;
+      int n_pg = 0;
+      bool bad = false;
+      if (n_my > 0) fetch(w, &page, &n_pg, &bad);
+      for (int i = 0; i < n_my; ++i) {
+        const int s = i % C::NSTAGE;
+        int64_t page_n = 0;
+        int n_pg_n = 0;
+        bool bad_n = false;
+        if (i + 1 < n_my) {
+          TileWalk wn = w;
+          wn.next(p);
+          fetch(wn, &page_n, &n_pg_n, &bad_n);
+        }
+        if (lane == 0) stage_wait(s, i);
+        if (__any_sync(kFull, bad)) {
+          if (lane == 0) {
+            atomicCAS(p.err, 0, kErrBadPage);
+            *abort_flag = 1;
+          }
+          break;
+        }
         const int64_t len = p.seq_len[w.b];
         const int64_t t0 = w.j * C::TILE;
         const int nv = static_cast<int>(min(static_cast<int64_t>(C::TILE), len - t0));
-        if (!(cta == 0 && i == p.debug_skip_tile)) {
-          const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
-          constexpr uint32_t q_bytes = G * D * C::ELEM;
-          const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
-          uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
-          mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
-          if (with_q) {
-            // One copy per query token of the launch: its `heads` query heads are contiguous.
-            const int heads = 1 << p.log2_heads;
-            const uint32_t qb = static_cast<uint32_t>(heads) * D * C::ELEM;
-            for (int jl = 0; jl < (G >> p.log2_heads); ++jl) {
-              const uint8_t* qsrc =
-                  reinterpret_cast<const uint8_t*>(p.q) +
-                  ((static_cast<int64_t>(w.b) * p.n_queries + p.q_first + jl) * p.n_q_heads + w.h * heads) * D *
-                      C::ELEM;
-              bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
-            }
+        const bool skip = (cta == 0 && i == p.debug_skip_tile);
+        bool go = false;
+        if (lane == 0) {
+          go = *abort_flag == 0;
+          if (go && !skip) {
+            tile_header(s, i, static_cast<uint32_t>(nv) * C::ROW);
+            ++fills[s];
           }
-          if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
-          if (bytes != 0) {
-            const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
-            bulk_load(sm.k[s], reinterpret_cast<const T*>(p.k) + off, bytes, &sm.full[s], pol);
-            bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, vbar, pol);
-          }
-          ++fills[s];
         }
+        if (!__shfl_sync(kFull, go, 0)) break;
+        if (!skip && lane < n_pg) {
+          const int64_t ps = int64_t(1) << p.log2_page;
+          const int64_t first = ((t0 >> p.log2_page) + lane) << p.log2_page;  // first token of the page
+          const int64_t lo = max(t0, first), hi = min(t0 + nv, first + ps);
+          const uint32_t nb = static_cast<uint32_t>(hi - lo) * C::ROW;
+          const int64_t row = ((page * p.n_kv_heads + w.h) << p.log2_page) + (lo - first);
+          bulk_load(sm.k[s] + (lo - t0) * C::ROW, reinterpret_cast<const T*>(p.k) + row * D, nb, &sm.full[s], pol);
+          bulk_load(sm.v[s] + (lo - t0) * C::ROW, reinterpret_cast<const T*>(p.v) + row * D, nb, &vbar0[s], pol);
+        }
+        page = page_n;
+        n_pg = n_pg_n;
+        bad = bad_n;
         w.next(p);
       }
-      // No copy may still be landing in shared memory when the CTA exits.
+    }
+    // No copy may still be landing in shared memory when the CTA exits.
+    if (lane == 0) {
 #pragma unroll
-      for (int s = 0; s < C::NSTAGE; ++s) {
-        if (fills[s] > 0 && !wait_phase(&sm.full[s], (fills[s] - 1) & 1, p.wait_limit_ns, nullptr))
+      for (int st = 0; st < C::NSTAGE; ++st) {
+        if (fills[st] > 0 && !wait_phase(&sm.full[st], (fills[st] - 1) & 1, p.wait_limit_ns, nullptr))
           atomicCAS(p.err, 0, kErrDrainWait);
-        if (TA_SPLIT_KV_BARRIERS && fills[s] > 0 &&
-            !wait_phase(&sm.full_v[s], (fills[s] - 1) & 1, p.wait_limit_ns, nullptr))
+        if (TA_SPLIT_KV_BARRIERS && fills[st] > 0 &&
+            !wait_phase(&sm.full_v[st], (fills[st] - 1) & 1, p.wait_limit_ns, nullptr))
           atomicCAS(p.err, 0, kErrDrainWait);
       }
     }

@@ -1,6 +1,6 @@
 // Host-side handle of the compiled split-KV kernel instances.  Each (element type, tile
-// configuration, head_dim) is compiled in a translation unit of its own
-// (split_kv_<type>_<tiles>_d<D>.cu) so that the instances build in parallel.
+// configuration, head_dim, contiguous or paged cache) is compiled in a translation unit of
+// its own (split_kv_[paged_]<type>_<tiles>_d<D>.cu) so that the instances build in parallel.
 #pragma once
 #include <cuda_bf16.h>
 
@@ -17,23 +17,31 @@ struct KernelInfo {
   int threads;
 };
 
-template <typename T, int D, int G, class V>
+template <typename T, int D, int G, class V, bool PAGED>
 KernelInfo make_info() {
   using C = SplitCfg<T, D, G, V>;
-  return KernelInfo{&split_kv_decode_kernel<T, D, G, V>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
+  return KernelInfo{&split_kv_decode_kernel<T, D, G, V, PAGED>, sizeof(SplitSmem<C>), C::TILE, C::THREADS};
 }
 
-// The instance for group size G (1, 2, 4 or 8) of one (T, V, D); false for any other G.
-template <typename T, class V, int D>
+// The instance for group size G (1, 2, 4 or 8) of one (T, V, D, PAGED); false for any other G.
+template <typename T, class V, int D, bool PAGED>
 bool split_instance(int G, KernelInfo* ki);
 
-template <> bool split_instance<__nv_bfloat16, LongTiles, 64>(int, KernelInfo*);
-template <> bool split_instance<__nv_bfloat16, LongTiles, 128>(int, KernelInfo*);
-template <> bool split_instance<__nv_bfloat16, ShortTiles, 64>(int, KernelInfo*);
-template <> bool split_instance<__nv_bfloat16, ShortTiles, 128>(int, KernelInfo*);
-template <> bool split_instance<float, LongTiles, 64>(int, KernelInfo*);
-template <> bool split_instance<float, LongTiles, 128>(int, KernelInfo*);
-template <> bool split_instance<float, ShortTiles, 64>(int, KernelInfo*);
-template <> bool split_instance<float, ShortTiles, 128>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, LongTiles, 64, false>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, LongTiles, 64, true>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, LongTiles, 128, false>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, LongTiles, 128, true>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, ShortTiles, 64, false>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, ShortTiles, 64, true>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, ShortTiles, 128, false>(int, KernelInfo*);
+template <> bool split_instance<__nv_bfloat16, ShortTiles, 128, true>(int, KernelInfo*);
+template <> bool split_instance<float, LongTiles, 64, false>(int, KernelInfo*);
+template <> bool split_instance<float, LongTiles, 64, true>(int, KernelInfo*);
+template <> bool split_instance<float, LongTiles, 128, false>(int, KernelInfo*);
+template <> bool split_instance<float, LongTiles, 128, true>(int, KernelInfo*);
+template <> bool split_instance<float, ShortTiles, 64, false>(int, KernelInfo*);
+template <> bool split_instance<float, ShortTiles, 64, true>(int, KernelInfo*);
+template <> bool split_instance<float, ShortTiles, 128, false>(int, KernelInfo*);
+template <> bool split_instance<float, ShortTiles, 128, true>(int, KernelInfo*);
 
 }  // namespace ta

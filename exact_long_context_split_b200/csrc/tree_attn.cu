@@ -33,20 +33,22 @@ ta_status cuda_fail(cudaError_t e) {
 // Kernel instances
 // ------------------------------------------------------------------------------------------
 
-template <class V>
+template <class V, bool PAGED>
 bool pick_variant(ta_dtype dt, int D, int G, KernelInfo* ki) {
   if (dt == TA_BF16) {
-    if (D == 64) return split_instance<__nv_bfloat16, V, 64>(G, ki);
-    if (D == 128) return split_instance<__nv_bfloat16, V, 128>(G, ki);
+    if (D == 64) return split_instance<__nv_bfloat16, V, 64, PAGED>(G, ki);
+    if (D == 128) return split_instance<__nv_bfloat16, V, 128, PAGED>(G, ki);
   } else if (dt == TA_F32) {
-    if (D == 64) return split_instance<float, V, 64>(G, ki);
-    if (D == 128) return split_instance<float, V, 128>(G, ki);
+    if (D == 64) return split_instance<float, V, 64, PAGED>(G, ki);
+    if (D == 128) return split_instance<float, V, 128, PAGED>(G, ki);
   }
   return false;
 }
 
-bool pick_kernel(ta_dtype dt, int D, int G, bool short_tiles, KernelInfo* ki) {
-  return short_tiles ? pick_variant<ShortTiles>(dt, D, G, ki) : pick_variant<LongTiles>(dt, D, G, ki);
+bool pick_kernel(ta_dtype dt, int D, int G, bool short_tiles, KernelInfo* ki, bool paged = false) {
+  if (paged)
+    return short_tiles ? pick_variant<ShortTiles, true>(dt, D, G, ki) : pick_variant<LongTiles, true>(dt, D, G, ki);
+  return short_tiles ? pick_variant<ShortTiles, false>(dt, D, G, ki) : pick_variant<LongTiles, false>(dt, D, G, ki);
 }
 
 // Tile configuration for a batch: short tiles when the mean (sequence, KV head) unit is
@@ -205,12 +207,20 @@ bool any_tokens(const int64_t* seqlens, int batch) {
 // Launch of a planned decode (workspace body at `body`, error word at `err`)
 // ------------------------------------------------------------------------------------------
 
+// A paged cache: pages [num_pages][Hkv][page_size][D], block table rows of `stride` entries.
+struct PagedCache {
+  const int32_t* table = nullptr;
+  int64_t stride = 0;
+  int64_t num_pages = 0;
+  int log2_page = 0;
+};
+
 // n_queries / q_first: query tokens per sequence and the first one this launch covers (the
 // kernel instance's G rows per unit are G / (Hq / Hkv) consecutive query tokens).
 ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, const void* k, const void* v,
                       float* out, float* lse, int Hq, int Hkv, int D, float scale, ta_dtype dt,
                       const ta_options* opts, uint8_t* body, int* err, cudaStream_t st, int n_queries = 1,
-                      int q_first = 0) {
+                      int q_first = 0, const PagedCache* pc = nullptr) {
   const size_t qe = (dt == TA_BF16) ? 2 : 4;
   int log2_heads = 0;
   while ((1 << (log2_heads + 1)) <= Hq / Hkv) ++log2_heads;
@@ -239,6 +249,12 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
     p.n_queries = n_queries;
     p.q_first = q_first;
     p.log2_heads = log2_heads;
+    if (pc) {
+      p.block_table = pc->table + static_cast<int64_t>(g.b0) * pc->stride;
+      p.bt_stride = pc->stride;
+      p.num_pages = pc->num_pages;
+      p.log2_page = pc->log2_page;
+    }
     for (int i = 0; i < g.nb; ++i) {
       p.kv_off[i] = g.kv_off[i];
       p.seq_len[i] = g.len[i];
@@ -702,6 +718,7 @@ const char* tree_attn_status_string(ta_status s) {
     case TA_ERR_CUDA: return "CUDA error";
     case TA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case TA_ERR_SCRATCH_LIMIT: return "needs more scratch than the fixed 4 MiB no-allocation buffer holds";
+    case TA_ERR_BAD_PAGE: return "a block-table entry is outside [0, num_pages)";
   }
   return "unknown status";
 }
@@ -895,6 +912,88 @@ ta_status tree_attn_decode_multi(const void* q, const void* k_cache, const void*
   return with_temp_workspace(kHeaderBytes + plan.body, static_cast<cudaStream_t>(stream), &multi_alloc_run, &ctx);
 }
 
+namespace {
+struct PagedArgs {
+  DecodeArgs a;
+  PagedCache pc;
+};
+
+ta_status paged_validate(const DecodeArgs& a, const PagedCache& pc, int32_t page_size, const ta_options* opts,
+                         bool check_pointers, KernelInfo* ki, PagedCache* out) {
+  if (page_size < 16 || page_size > 65536 || (page_size & (page_size - 1)) != 0) return TA_ERR_INVALID_ARG;
+  if (pc.num_pages < 0) return TA_ERR_INVALID_ARG;
+  *out = pc;
+  out->log2_page = 0;
+  while ((1 << out->log2_page) < page_size) ++out->log2_page;
+  ta_status s = validate(a, opts, check_pointers, ki);
+  if (s != TA_OK) return s;
+  pick_kernel(a.dt, a.D, a.Hq / a.Hkv, use_short_tiles(a.seqlens, a.batch, opts), ki, true);
+  int64_t max_blocks = 0;
+  for (int b = 0; b < a.batch; ++b) max_blocks = std::max<int64_t>(max_blocks, (a.seqlens[b] + page_size - 1) / page_size);
+  if (max_blocks > 0 && (pc.stride < max_blocks || pc.num_pages < 1)) return TA_ERR_INVALID_ARG;
+  // A tile touches at most tile / page_size + 1 pages, one producer lane each.
+  if (ki->tile / page_size + 1 > 32) return TA_ERR_UNSUPPORTED;
+  if (check_pointers && max_blocks > 0 && (!pc.table || (reinterpret_cast<uintptr_t>(pc.table) & 3) != 0))
+    return TA_ERR_INVALID_ARG;
+  return TA_OK;
+}
+
+ta_status paged_run(const PagedArgs& pa, const ta_options* opts, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const DecodeArgs& a = pa.a;
+  KernelInfo ki;
+  PagedCache pc;
+  ta_status s = paged_validate(a, pa.pc, 1 << pa.pc.log2_page, opts, true, &ki, &pc);
+  if (s != TA_OK) return s;
+  if (a.batch == 0) return TA_OK;
+  if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
+  Plan plan;
+  s = plan_for(a, opts, ki, &plan);
+  if (s != TA_OK) return s;
+  if (ws_bytes < kHeaderBytes + plan.body_bytes) return TA_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return launch_plan(plan, ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt, opts,
+                     base + kHeaderBytes, reinterpret_cast<int*>(base), st, 1, 0, &pc);
+}
+
+ta_status paged_alloc_run(void* ws, size_t bytes, void* ctx, cudaStream_t st) {
+  return paged_run(*static_cast<PagedArgs*>(ctx), nullptr, ws, bytes, st);
+}
+}  // namespace
+
+ta_status tree_attn_decode_paged_ex(ta_dtype dtype, const void* q, const void* k_pages, const void* v_pages,
+                                    int64_t num_pages, int32_t page_size, const int32_t* block_table,
+                                    int64_t block_table_stride, const int64_t* seqlens, int32_t batch,
+                                    int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale, float* out,
+                                    float* lse, const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  PagedArgs pa{DecodeArgs{dtype, q, k_pages, v_pages, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+                          scale, out, lse},
+               PagedCache{block_table, block_table_stride, num_pages, 0}};
+  if (page_size < 16 || (page_size & (page_size - 1)) != 0) return TA_ERR_INVALID_ARG;
+  while ((1 << pa.pc.log2_page) < page_size) ++pa.pc.log2_page;
+  return paged_run(pa, opts, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                                 int32_t page_size, const int32_t* block_table, int64_t block_table_stride,
+                                 const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int32_t head_dim, float scale, float* out, float* lse, void* stream) {
+  PagedArgs pa{DecodeArgs{TA_BF16, q, k_pages, v_pages, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+                          scale, out, lse},
+               PagedCache{block_table, block_table_stride, num_pages, 0}};
+  if (page_size < 16 || (page_size & (page_size - 1)) != 0) return TA_ERR_INVALID_ARG;
+  while ((1 << pa.pc.log2_page) < page_size) ++pa.pc.log2_page;
+  KernelInfo ki;
+  PagedCache pc;
+  ta_status s = paged_validate(pa.a, pa.pc, page_size, nullptr, true, &ki, &pc);
+  if (s != TA_OK || batch == 0) return s;
+  Plan plan;
+  s = plan_for(pa.a, nullptr, ki, &plan);
+  if (s != TA_OK) return s;
+  return with_temp_workspace(kHeaderBytes + plan.body_bytes, static_cast<cudaStream_t>(stream), &paged_alloc_run,
+                             &pa);
+}
+
 // ------------------------------------------------------------------------------------------
 // Decode without allocation: the workspace is a fixed array in the library's device memory.
 // ------------------------------------------------------------------------------------------
@@ -967,7 +1066,8 @@ ta_status tree_attn_check(const void* ws, void* stream) {
   int word = 0;
   e = cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
-  return word == 0 ? TA_OK : TA_ERR_TIMEOUT;
+  if (word == 0) return TA_OK;
+  return word == kErrBadPage ? TA_ERR_BAD_PAGE : TA_ERR_TIMEOUT;
 }
 
 }  // extern "C"

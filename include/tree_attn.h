@@ -67,7 +67,9 @@ typedef enum {
   TA_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than required */
   TA_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed; see tree_attn_last_cuda_error() */
   TA_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out (reported by tree_attn_check) */
-  TA_ERR_SCRATCH_LIMIT = 6 /* tree_attn_decode_noalloc: the problem needs more scratch than its fixed buffer */
+  TA_ERR_SCRATCH_LIMIT = 6, /* tree_attn_decode_noalloc: the problem needs more scratch than its fixed buffer */
+  TA_ERR_BAD_PAGE = 7       /* paged decode: a block-table entry outside [0, num_pages) (reported by
+                               tree_attn_check; nothing was read through it, the outputs are NaN) */
 } ta_status;
 
 typedef enum { TA_BF16 = 0, TA_F32 = 1 } ta_dtype;
@@ -229,9 +231,39 @@ ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const voi
                                    float scale, float* out, float* lse, void* stream);
 
 /*
+ * Decode over a paged KV cache, after the attention-acceleration concept page
+ * (compassingai.com, part 3 "PagedAttention (vLLM)"): the cache is cut into blocks of
+ * `page_size` tokens, and a table maps each sequence's logical blocks to physical ones, which
+ * sequences may share (a common prompt prefix, for example).
+ *   k_pages, v_pages  [num_pages][Hkv][page_size][D] (bf16, or f32 with TA_F32): physical block
+ *                     p holds page_size consecutive token rows of every KV head
+ *   block_table       DEVICE int32 [B][block_table_stride]: sequence b's tokens
+ *                     [i * page_size, (i + 1) * page_size) are rows 0.. of physical block
+ *                     block_table[b * block_table_stride + i]; stride >= ceil(max S_b / page_size)
+ *   page_size         a power of two >= 16 (TA_ERR_INVALID_ARG otherwise)
+ * q, out, lse, seqlens, workspace (tree_attn_workspace_size applies unchanged) and the other
+ * rules as tree_attn_decode_ex.  Every entry a sequence uses is checked against num_pages on
+ * the device before anything is read through it: an entry outside [0, num_pages) makes
+ * tree_attn_check report TA_ERR_BAD_PAGE and the affected outputs NaN.
+ */
+ta_status tree_attn_decode_paged_ex(ta_dtype dtype, const void* q, const void* k_pages, const void* v_pages,
+                                    int64_t num_pages, int32_t page_size, const int32_t* block_table,
+                                    int64_t block_table_stride, const int64_t* seqlens, int32_t batch,
+                                    int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale, float* out,
+                                    float* lse, const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/* Paged decode, bf16, allocating its workspace per call like tree_attn_decode. */
+ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
+                                 int32_t page_size, const int32_t* block_table, int64_t block_table_stride,
+                                 const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
+                                 int32_t head_dim, float scale, float* out, float* lse, void* stream);
+
+/*
  * Synchronise `stream` and read the workspace's error word: TA_OK, or
  * TA_ERR_TIMEOUT if a kernel's bounded wait ran out since the workspace was
- * last initialised (the affected outputs are NaN), or TA_ERR_CUDA.
+ * last initialised (the affected outputs are NaN), TA_ERR_BAD_PAGE (paged decode, above),
+ * or TA_ERR_CUDA.
  */
 ta_status tree_attn_check(const void* workspace, void* stream);
 

@@ -29,7 +29,7 @@ _SRC = os.path.join(_HERE, "gen.c")
 _LIB = os.path.join(_HERE, "libsynth.so")
 
 # Tensor ids of the counter-based streams.
-TID_Q, TID_K, TID_V, TID_SPIKE, TID_K_SUFFIX, TID_V_SUFFIX = 0, 1, 2, 3, 4, 5
+TID_Q, TID_K, TID_V, TID_SPIKE, TID_K_SUFFIX, TID_V_SUFFIX, TID_PAGES = 0, 1, 2, 3, 4, 5, 6
 
 
 def build(force: bool = False) -> str:
@@ -126,6 +126,7 @@ class DecodeSpec:
     spike_factor: float = 4.0
     scale_value: Optional[float] = None  # softmax scale; default 1/sqrt(head_dim) rounded to float32
     n_queries: int = 1
+    page_size: int = 0  # > 0: the cache is paged (blocks of page_size tokens, seeded placement)
 
     @property
     def batch(self) -> int:
@@ -246,6 +247,44 @@ def make_decode_inputs(spec: DecodeSpec) -> Dict[str, np.ndarray]:
         "seqlens": np.asarray(spec.seqlens, dtype=np.int64),
         "spikes": spikes,
     }
+
+
+def page_table(seed: int, seqlens: Sequence[int], page_size: int, spare: int = 0):
+    """Block table placing each logical block of each sequence in a distinct physical block, in a
+    seeded random order, with `spare` physical blocks left unused.  Returns (table [B][max
+    blocks] int32, number of physical blocks)."""
+    blocks = [-(-int(S) // page_size) for S in seqlens]
+    n = sum(blocks) + spare
+    perm = np.random.default_rng([seed, TID_PAGES]).permutation(n).astype(np.int32)
+    table = np.zeros((len(seqlens), max([1] + blocks)), dtype=np.int32)
+    used = 0
+    for b, nb in enumerate(blocks):
+        table[b, :nb] = perm[used:used + nb]
+        used += nb
+    return table, n
+
+
+def scatter_pages(cache, seqlens: Sequence[int], n_kv_heads: int, head_dim: int, page_size: int, table,
+                  num_pages: int, fill):
+    """Lay a packed cache ([Hkv][S_b][D] blocks back to back) out as physical blocks
+    [num_pages][Hkv][page_size][D] through `table`; rows no token maps to hold `fill`."""
+    Hkv, D, ps = n_kv_heads, head_dim, page_size
+    pages = np.full((num_pages, Hkv, ps, D), fill, dtype=cache.dtype)
+    off = 0
+    for b, S in enumerate(seqlens):
+        S = int(S)
+        blk = cache[off:off + Hkv * S * D].reshape(Hkv, S, D)
+        off += Hkv * S * D
+        for i in range(-(-S // ps)):
+            n = min(ps, S - i * ps)
+            pages[table[b, i], :, :n, :] = blk[:, i * ps:i * ps + n, :]
+    return pages
+
+
+def paged_configs() -> Dict[str, DecodeSpec]:
+    """long_1m's cache in 16-token blocks placed at random (the common serving block size)."""
+    return {"long_1m_paged": DecodeSpec("long_1m_paged", [1_048_576], 32, 8, 128, seed=3, spike_frac=0.001,
+                                        page_size=16)}
 
 
 def make_bifurcated_inputs(spec: BifurcatedSpec) -> Dict[str, np.ndarray]:

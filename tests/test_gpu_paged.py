@@ -1,0 +1,169 @@
+"""GPU parity of decode over a paged KV cache (block table) against the CPU oracle, through
+the C ABI.  Unused page rows hold NaN, so any read through a wrong entry shows up."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import compare, decode_gpu, device_tensor, new_workspace
+
+pytestmark = pytest.mark.gpu
+
+NAN = {"bf16": np.uint16(0x7FC0), "f32": np.float32("nan")}
+
+
+def paged_case(seqlens, Hq, Hkv, D, dtype, ps, seed, spare=3):
+    sp = synth.DecodeSpec("paged", list(seqlens), Hq, Hkv, D, dtype=dtype, seed=seed)
+    inp = synth.make_decode_inputs(sp)
+    table, n_pages = synth.page_table(seed, seqlens, ps, spare=spare)
+    kp = synth.scatter_pages(inp["k"], seqlens, Hkv, D, ps, table, n_pages, NAN[dtype])
+    vp = synth.scatter_pages(inp["v"], seqlens, Hkv, D, ps, table, n_pages, NAN[dtype])
+    return sp, inp, table, n_pages, kp, vp
+
+
+def paged_gpu(sp, inp, table, n_pages, kp, vp, ps, opts=None, entry="ex", expect=None):
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    B, Hq, Hkv, D = sp.batch, sp.n_q_heads, sp.n_kv_heads, sp.head_dim
+    q = device_tensor(inp["q"], sp.dtype)
+    k = device_tensor(kp.reshape(-1), sp.dtype)
+    v = device_tensor(vp.reshape(-1), sp.dtype)
+    bt = torch.from_numpy(np.ascontiguousarray(table)).cuda()
+    out = torch.full((B, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((B, Hq), float("nan"), device="cuda")
+    lens = [int(s) for s in sp.seqlens]
+    if entry == "ex":
+        ws = new_workspace(ta.tree_attn_workspace_size(lens, Hq, Hkv, D, sp.dtype, opts))
+        ta.tree_attn_decode_paged_ex(sp.dtype, q, k, v, n_pages, ps, bt, table.shape[1], lens, Hq, Hkv, D, sp.scale,
+                                     out, lse, opts, ws)
+        status = ta.tree_attn_check(ws)
+        assert status == (ta.TA_OK if expect is None else expect), ta.tree_attn_status_string(status)
+    else:
+        ta.tree_attn_decode_paged(q, k, v, n_pages, ps, bt, table.shape[1], lens, Hq, Hkv, D, sp.scale, out, lse)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def oracle_paged(sp, inp, table, kp, vp, ps, pairs=None):
+    return oracle.paged_decode_attention(inp["q"], kp.reshape(-1), vp.reshape(-1), table, sp.seqlens, ps,
+                                         sp.n_q_heads, sp.n_kv_heads, sp.head_dim, sp.scale, dtype=sp.dtype,
+                                         pairs=pairs)
+
+
+CASES = [
+    ([1, 0, 17, 33, 64, 200, 1000, 3001], 8, 2, 128, "bf16", 16),
+    ([5, 129, 2049], 4, 4, 64, "bf16", 32),
+    ([300, 20000], 32, 4, 128, "bf16", 256),
+    ([100, 4097], 8, 2, 64, "f32", 64),
+    ([1024, 5, 1500], 16, 4, 128, "bf16", 1024),
+]
+
+
+@pytest.mark.parametrize("tiles", [1, 2])
+@pytest.mark.parametrize("case", CASES, ids=[f"ps{c[5]}_G{c[1] // c[2]}_D{c[3]}_{c[4]}" for c in CASES])
+def test_paged_against_oracle(case, tiles):
+    import exact_long_context_split_b200 as ta
+
+    seqlens, Hq, Hkv, D, dtype, ps = case
+    sp, inp, table, n_pages, kp, vp = paged_case(seqlens, Hq, Hkv, D, dtype, ps, seed=50 + ps + D)
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, ps, ta.make_options(split_tiles=tiles))
+    ref_out, ref_lse = oracle_paged(sp, inp, table, kp, vp, ps)
+    compare(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("num_ctas", [1, 7, 148, 100000])
+def test_paged_bit_identical_to_contiguous(num_ctas):
+    """The paged layout changes where tiles come from, not what is computed."""
+    import exact_long_context_split_b200 as ta
+
+    seqlens = [5000, 77, 0, 2100]
+    sp, inp, table, n_pages, kp, vp = paged_case(seqlens, 16, 4, 128, "bf16", 16, seed=5)
+    opts = ta.make_options(num_ctas=num_ctas)
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, 16, opts)
+    ref_out, ref_lse = decode_gpu(inp, sp, opts)
+    assert np.array_equal(out.view(np.uint32), ref_out.view(np.uint32))
+    assert np.array_equal(lse.view(np.uint32), ref_lse.view(np.uint32))
+
+
+def test_shared_prefix_blocks():
+    """Two sequences whose tables share their first blocks (a common prompt prefix)."""
+    seqlens = [160, 100]
+    sp, inp, table, n_pages, kp, vp = paged_case(seqlens, 8, 2, 128, "bf16", 32, seed=8)
+    table = table.copy()
+    table[1, :3] = table[0, :3]  # sequence 1 reads sequence 0's first 96 tokens
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, 32)
+    ref_out, ref_lse = oracle_paged(sp, inp, table, kp, vp, 32)
+    compare(out, lse, ref_out, ref_lse)
+
+
+def test_allocating_entry_point():
+    sp, inp, table, n_pages, kp, vp = paged_case([300, 5, 1000], 8, 2, 128, "bf16", 16, seed=9)
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, 16, entry="alloc")
+    ref_out, ref_lse = oracle_paged(sp, inp, table, kp, vp, 16)
+    compare(out, lse, ref_out, ref_lse)
+
+
+def test_bad_block_table_entry_is_reported():
+    """An entry outside [0, num_pages) is caught on the device before any read through it: the
+    call reports TA_ERR_BAD_PAGE, the poisoned rows are NaN, and the next call succeeds."""
+    import exact_long_context_split_b200 as ta
+
+    seqlens = [300, 70]
+    sp, inp, table, n_pages, kp, vp = paged_case(seqlens, 8, 2, 128, "bf16", 16, seed=10, spare=0)
+    bad = table.copy()
+    bad[0, 5] = n_pages  # one past the last physical block
+    out, lse = paged_gpu(sp, inp, bad, n_pages, kp, vp, 16, expect=ta.TA_ERR_BAD_PAGE)
+    assert np.isnan(out[0]).all() and np.isnan(lse[0]).all()
+    bad[0, 5] = -1
+    paged_gpu(sp, inp, bad, n_pages, kp, vp, 16, expect=ta.TA_ERR_BAD_PAGE)
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, 16)
+    ref_out, ref_lse = oracle_paged(sp, inp, table, kp, vp, 16)
+    compare(out, lse, ref_out, ref_lse)
+
+
+def test_invalid_page_size():
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    z = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(8, dtype=torch.int32, device="cuda")
+    o = torch.empty(8 * 128, device="cuda")
+    for ps in (8, 24, 0):
+        with pytest.raises(ta.TreeAttnError) as e:
+            ta.tree_attn_decode_paged(z, z, z, 1, ps, bt, 8, [5], 8, 2, 128, 0.1, o, o)
+        assert e.value.status == ta.TA_ERR_INVALID_ARG
+
+
+def test_long_1m_paged_sampled():
+    """The bench workload: 1M tokens in 16-token blocks at random places, sampled rows."""
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    sp = synth.paged_configs()["long_1m_paged"]
+    inp = synth.make_decode_inputs(sp)
+    S, Hkv, D, ps = sp.seqlens[0], sp.n_kv_heads, sp.head_dim, sp.page_size
+    table, n_pages = synth.page_table(sp.seed, sp.seqlens, ps)
+    bt = torch.from_numpy(table).cuda()
+    idx = bt[0].long()
+    pages = {}
+    for name in ("k", "v"):
+        c = device_tensor(inp[name], "bf16").view(Hkv, S // ps, ps, D).permute(1, 0, 2, 3)
+        pg = torch.empty(n_pages, Hkv, ps, D, dtype=torch.bfloat16, device="cuda")
+        pg[idx] = c
+        pages[name] = pg
+    q = device_tensor(inp["q"], "bf16")
+    out = torch.empty(1, 32, D, device="cuda")
+    lse = torch.empty(1, 32, device="cuda")
+    ws = new_workspace(ta.tree_attn_workspace_size([S], 32, Hkv, D))
+    ta.tree_attn_decode_paged_ex("bf16", q, pages["k"], pages["v"], n_pages, ps, bt, table.shape[1], [S], 32, Hkv, D,
+                                 sp.scale, out, lse, None, ws)
+    assert ta.tree_attn_check(ws) == ta.TA_OK
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    pairs = [(0, 0), (0, 13), (0, 31)]
+    ref_out, ref_lse = oracle.decode_attention(inp["q"], inp["k"], inp["v"], sp.seqlens, 32, Hkv, D, sp.scale,
+                                               pairs=pairs)
+    compare(out, lse, ref_out, ref_lse, pairs=pairs)
