@@ -17,11 +17,13 @@ from .attention import (  # noqa: F401
     finalize,
     gather_paged_sequence,
     merge,
+    merge_shard_results,
     merge_tree,
     multi_query_attention,
     online_softmax,
     paged_decode_attention,
     sequence_block,
+    shard_bounds,
     split_attention,
     to_f64,
 )

@@ -51,6 +51,11 @@ design notes):
    (which sequences may share).  Layout read here: physical block p holds, for each KV head
    h, page_size consecutive token rows [p][h][0..page_size)[D]; logical block i of sequence b
    (its tokens i * page_size ...) is physical block table[b][i].
+9. Sequence-sharded decode ([TreeAttn], tree all-reduce across devices; [StarAttn] phase 2,
+   the query host combining the hosts' softmax statistics): device r holds the contiguous
+   token range shard_bounds(S, W, r) of every sequence and computes ordinary decode attention
+   over it, i.e. (out_r, lse_r); the results combine exactly as partials (m = lse_r, l = 1,
+   o = out_r) merged in a fixed pairwise tree over r.  A shard with no token gives (0, -inf).
 """
 from __future__ import annotations
 
@@ -364,3 +369,18 @@ def paged_decode_attention(q, k_pages, v_pages, block_table, seqlens: Sequence[i
     blocks = [gather_paged_sequence(v_pages, block_table[b], seqlens[b], Hkv, page_size, D) for b in range(B)]
     vc = np.concatenate([x.reshape(-1) for x in blocks]) if B else np.zeros(0, dtype=np.asarray(v_pages).dtype)
     return decode_attention(q, kc, vc, seqlens, n_q_heads, n_kv_heads, head_dim, scale, dtype=dtype, pairs=pairs)
+
+
+def shard_bounds(seqlen: int, n_shards: int, shard: int) -> Tuple[int, int]:
+    """Token range [t0, t1) of shard `shard` of n_shards contiguous shards of a sequence
+    (reading 9): t0 = floor(shard * S / n), t1 = floor((shard + 1) * S / n)."""
+    S = int(seqlen)
+    return shard * S // n_shards, (shard + 1) * S // n_shards
+
+
+def merge_shard_results(outs, lses):
+    """Combine the (out, lse) of every shard of one row (reading 9): each is the partial
+    (lse, 1, out) in natural-log units; a fixed pairwise tree over the shards, then finalize."""
+    parts = [(float(l), 1.0 if l != -math.inf else 0.0, np.asarray(o, dtype=np.float64) if l != -math.inf
+              else np.zeros_like(np.asarray(o, dtype=np.float64))) for o, l in zip(outs, lses)]
+    return finalize(merge_tree(parts))

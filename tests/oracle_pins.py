@@ -500,6 +500,36 @@ def pin_paged_cache(O):
     _close(g1[:, :ps], g0[:, :ps], rtol=0.0, what="shared block")
 
 
+def pin_sharded_decode(O):
+    """[TreeAttn] across devices (reading 9): a cache cut into W contiguous shards (some empty),
+    each shard's own attention (out, lse) merged by merge_shard_results equals the textbook
+    attention over the whole cache; the shard bounds tile [0, S) exactly."""
+    r = _rng(27)
+    D = 5
+    for S, W in ((11, 3), (3, 4), (16, 8), (1, 2)):
+        bounds = [O.shard_bounds(S, W, i) for i in range(W)]
+        assert bounds[0][0] == 0 and bounds[-1][1] == S
+        assert all(bounds[i][1] == bounds[i + 1][0] for i in range(W - 1))
+        K = r.standard_normal((S, D))
+        V = r.standard_normal((S, D))
+        q = r.standard_normal(D)
+        outs, lses = [], []
+        for t0, t1 in bounds:
+            x = 0.9 * (K[t0:t1] @ q)
+            if t1 == t0:
+                outs.append(np.zeros(D))
+                lses.append(-math.inf)
+                continue
+            e = np.exp(x - x.max())
+            outs.append((e @ V[t0:t1]) / e.sum())
+            lses.append(x.max() + math.log(e.sum()))
+        out, lse = O.merge_shard_results(outs, lses)
+        x = 0.9 * (K @ q)
+        e = np.exp(x - x.max())
+        _close(out, (e @ V) / e.sum(), rtol=1e-12, atol=1e-14, what=f"sharded out S={S} W={W}")
+        _close(lse, x.max() + math.log(e.sum()), rtol=1e-13, what=f"sharded lse S={S} W={W}")
+
+
 ALL_PINS = [
     pin_bf16_decoding,
     pin_identical_keys,
@@ -521,4 +551,5 @@ ALL_PINS = [
     pin_long_cache_pieces,
     pin_multi_query,
     pin_paged_cache,
+    pin_sharded_decode,
 ]

@@ -38,6 +38,8 @@ MUTANTS = {
     "multi-query mask reversed": ("            visible = S - n + j + 1\n", "            visible = S - j\n"),
     "paged block index off by one": ("pages[int(block_row[t // ps]), :, t % ps, :]", "pages[int(block_row[t // ps + (t >= ps)]), :, t % ps, :]"),
     "paged rows ignore the head": ("pages[int(block_row[t // ps]), :, t % ps, :]", "pages[int(block_row[t // ps]), :1, t % ps, :]"),
+    "shard bounds overlap": ("    return shard * S // n_shards, (shard + 1) * S // n_shards", "    return shard * S // n_shards, min(S, (shard + 1) * S // n_shards + 1)"),
+    "shard merge ignores lse": ("    parts = [(float(l), 1.0 if l != -math.inf", "    parts = [(0.0 if l != -math.inf else l, 1.0 if l != -math.inf"),
     "pieces skip last rows": ("        acc += e[r0:r1] @ to_f64(Vbits[r0:r1], dtype)", "        acc += e[r0:r1 - (r1 == S)] @ to_f64(Vbits[r0:r1 - (r1 == S)], dtype)"),
 }
 
