@@ -38,6 +38,7 @@ EXPORTED = [
     "tree_attn_decode_multi",
     "tree_attn_decode_paged_ex",
     "tree_attn_decode_paged",
+    "tree_attn_merge_shards",
 ]
 
 
@@ -118,6 +119,7 @@ def lib() -> ctypes.CDLL:
                 [ctypes.c_int, vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, popt, vp, sz, vp],
                 ctypes.c_int,
             ),
+            "tree_attn_merge_shards": ([vp, vp, i32, i64, i32, vp, vp, vp], ctypes.c_int),
             "tree_attn_decode_paged": (
                 [vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
@@ -314,3 +316,9 @@ def tree_attn_decode_paged(q, k_pages, v_pages, num_pages, page_size, block_tabl
                                         _ptr(block_table), block_table_stride, arr, n, n_q_heads, n_kv_heads,
                                         head_dim, scale, _ptr(out), _ptr(lse), _stream(stream, q, out)),
            "tree_attn_decode_paged")
+
+
+def tree_attn_merge_shards(outs, lses, n_shards, rows, head_dim, out, lse, stream=None) -> None:
+    """Merge (out, lse) computed over n_shards slices of every sequence: outs [n_shards][rows][D]."""
+    _check(lib().tree_attn_merge_shards(_ptr(outs), _ptr(lses), n_shards, rows, head_dim, _ptr(out), _ptr(lse),
+                                        _stream(stream, outs, out)), "tree_attn_merge_shards")

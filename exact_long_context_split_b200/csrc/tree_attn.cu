@@ -512,6 +512,40 @@ __global__ void merge_two_kernel(const float* __restrict__ out_a, const float* _
   if (d == 0) lse[r] = l;
 }
 
+// Sequence-sharded results: out = sum_s w_s out_s / sum_s w_s, w_s = e^(lse_s - M),
+// lse = M + ln sum_s w_s, both sums over the shards in a fixed pairwise tree (a binary
+// counter over the shard index).  One thread per output element.
+__global__ void merge_shards_kernel(const float* __restrict__ outs, const float* __restrict__ lses, int n_shards,
+                                    int64_t rows, int D, float* __restrict__ out, float* __restrict__ lse) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= rows * D) return;
+  const int64_t r = i / D;
+  const int d = static_cast<int>(i % D);
+  float M = -INFINITY;
+  bool nan = false;
+  for (int sh = 0; sh < n_shards; ++sh) {
+    const float l = lses[sh * rows + r];
+    nan |= (l != l);
+    M = fmaxf(M, l);
+  }
+  PairwiseSum so, sw;
+  for (int sh = 0; sh < n_shards; ++sh) {
+    const float l = lses[sh * rows + r];
+    const float w = (l == -INFINITY) ? 0.f : expf(l - M);
+    sw.push(w);
+    so.push(w * outs[(sh * rows + r) * D + d]);
+  }
+  const float W = sw.result();
+  float o = 0.f, lv = -INFINITY;
+  if (W > 0.f) {
+    o = so.result() / W;
+    lv = M + logf(W);
+  }
+  if (nan) o = lv = __int_as_float(0x7fc00000);
+  out[i] = o;
+  if (d == 0) lse[r] = lv;
+}
+
 struct BifArgs {
   const void *q, *kp, *vp, *ks, *vs;
   int64_t P;
@@ -1057,6 +1091,20 @@ ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const voi
   if (e != cudaSuccess) return cuda_fail(e);
   return launch_plan(plan, ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt, nullptr,
                      base + kHeaderBytes, reinterpret_cast<int*>(base), st);
+}
+
+ta_status tree_attn_merge_shards(const float* outs, const float* lses, int32_t n_shards, int64_t rows,
+                                 int32_t head_dim, float* out, float* lse, void* stream) {
+  if (n_shards < 1 || n_shards > 65536 || rows < 0 || head_dim <= 0) return TA_ERR_INVALID_ARG;
+  if (rows == 0) return TA_OK;
+  if (!outs || !lses || !out || !lse) return TA_ERR_INVALID_ARG;
+  if (!aligned(outs, 4) || !aligned(lses, 4) || !aligned(out, 4) || !aligned(lse, 4)) return TA_ERR_INVALID_ARG;
+  const int64_t n = rows * head_dim;
+  merge_shards_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      outs, lses, n_shards, rows, head_dim, out, lse);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return TA_OK;
 }
 
 ta_status tree_attn_check(const void* ws, void* stream) {

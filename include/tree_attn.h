@@ -260,6 +260,25 @@ ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void*
                                  int32_t head_dim, float scale, float* out, float* lse, void* stream);
 
 /*
+ * Merge of sequence-sharded decode results, after the Tree Attention article (m.srwj168.com.cn,
+ * "The energy view of attention": max and logsumexp are associative, so the pieces each
+ * device computes over its slice of the cache combine exactly, in any order; across devices,
+ * a tree all-reduce) and the query host of Star Attention's phase 2.  Given the (out_s, lse_s)
+ * that a tree_attn_decode* call computed over shard s of every sequence's cache (the same
+ * rows in every shard), writes the result over the whole cache:
+ *   out = sum_s w_s out_s / sum_s w_s,  w_s = exp(lse_s - max_s lse_s),  lse = max + ln sum_s w_s
+ * with both sums over s in a fixed pairwise tree (bit-identical across calls).  A shard whose
+ * lse is -inf (no token) contributes nothing; all shards empty give out = 0, lse = -inf; a NaN
+ * lse in any shard gives NaN.
+ *   outs  DEVICE f32 [n_shards][rows][head_dim]    lses  DEVICE f32 [n_shards][rows]
+ *   out   DEVICE f32 [rows][head_dim]              lse   DEVICE f32 [rows]
+ * rows = B * Hq (times n for multi-query results); 1 <= n_shards <= 65536, else
+ * TA_ERR_INVALID_ARG.  No workspace; asynchronous on `stream`.
+ */
+ta_status tree_attn_merge_shards(const float* outs, const float* lses, int32_t n_shards, int64_t rows,
+                                 int32_t head_dim, float* out, float* lse, void* stream);
+
+/*
  * Synchronise `stream` and read the workspace's error word: TA_OK, or
  * TA_ERR_TIMEOUT if a kernel's bounded wait ran out since the workspace was
  * last initialised (the affected outputs are NaN), TA_ERR_BAD_PAGE (paged decode, above),

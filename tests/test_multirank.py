@@ -71,3 +71,73 @@ def test_record_fields():
         assert key in rec
     assert rec["scaling"] == "weak" and rec["config"]["workload"] == "long_1m"
     json.dumps(rec)
+
+
+def _sharded_rank(rank, world, port, q):
+    """One CPU rank of the sharded decode: the oracle stands in for the GPU decode and merge
+    (test infrastructure), so what runs here is the library's sharding plan and exchange."""
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    import oracle
+    import synth
+    from exact_long_context_split_b200.sharded import decode_sharded, shard_bounds
+
+    sp = synth.DecodeSpec("sharded", [37, 5, 1, 300], 8, 2, 16, dtype="f32", seed=12)
+    inp = synth.make_decode_inputs(sp)
+    Hkv, D = 2, 16
+    shard_lens, ks, vs, off = [], [], [], 0
+    for S in sp.seqlens:
+        t0, t1 = shard_bounds(S, world, rank)
+        shard_lens.append(t1 - t0)
+        ks.append(inp["k"][off:off + Hkv * S * D].reshape(Hkv, S, D)[:, t0:t1].reshape(-1))
+        vs.append(inp["v"][off:off + Hkv * S * D].reshape(Hkv, S, D)[:, t0:t1].reshape(-1))
+        off += Hkv * S * D
+
+    def decode(dtype, qq, k, v, lens, Hq, Hkv_, D_, scale, out, lse):
+        o, l = oracle.decode_attention(qq, k, v, lens, Hq, Hkv_, D_, scale, dtype=dtype)
+        out.copy_(torch.from_numpy(o.reshape(-1)))
+        lse.copy_(torch.from_numpy(l.reshape(-1)))
+
+    def merge(outs, lses, n, rows, D_, out, lse):
+        o = outs.numpy().reshape(n, rows, D_)
+        l = lses.numpy().reshape(n, rows)
+        res = [oracle.merge_shard_results(o[:, r], l[:, r]) for r in range(rows)]
+        out.view(-1).copy_(torch.from_numpy(np.stack([x[0] for x in res]).reshape(-1)))
+        lse.view(-1).copy_(torch.tensor([x[1] for x in res], dtype=torch.float64))
+
+    out = torch.empty(sp.batch, 8, D)
+    lse = torch.empty(sp.batch, 8)
+    decode_sharded(inp["q"], np.concatenate(ks), np.concatenate(vs), shard_lens, 8, Hkv, D, sp.scale, out, lse,
+                   dtype="f32", decode=decode, merge=merge)
+    ref_out, ref_lse = oracle.decode_attention(inp["q"], inp["k"], inp["v"], sp.seqlens, 8, Hkv, D, sp.scale,
+                                               dtype="f32")
+    err = float(np.max(np.abs(out.numpy() - ref_out)))
+    lerr = float(np.max(np.abs(lse.numpy() - ref_lse)))
+    q.put((rank, err, lerr, shard_lens))
+    dist.destroy_process_group()
+
+
+def test_sharded_decode_exchange_gloo():
+    """Two and three CPU ranks, each holding a contiguous slice of every sequence (one sequence
+    shorter than the rank count), exchange and merge to the unsharded result."""
+    for world in (2, 3):
+        ctx = mp.get_context("spawn")
+        q = ctx.Queue()
+        port = _free_port()
+        procs = [ctx.Process(target=_sharded_rank, args=(r, world, port, q)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(180)
+            assert p.exitcode == 0
+        res = sorted(q.get(timeout=5) for _ in range(world))
+        assert sum(r[3][2] for r in res) == 1  # the 1-token sequence lives on one rank only
+        for rank, err, lerr, _ in res:
+            assert err < 1e-5 and lerr < 1e-5, (world, rank, err, lerr)
