@@ -301,7 +301,7 @@ class DecodeRun:
         ta.tree_attn_workspace_init(self.ws)
         self.kv_bytes = spec.kv_bytes
         self.tokens = spec.tokens
-        self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv}>"
+        self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv},{'ShortTiles' if sum(self.seqlens) < 1024 * len(self.seqlens) else 'LongTiles'}>"
 
     def step(self, stream):
         sp = self.spec
