@@ -39,6 +39,7 @@ EXPORTED = [
     "tree_attn_decode_paged_ex",
     "tree_attn_decode_paged",
     "tree_attn_merge_shards",
+    "tree_attn_decode_multi_paged_ex",
 ]
 
 
@@ -120,6 +121,11 @@ def lib() -> ctypes.CDLL:
                 ctypes.c_int,
             ),
             "tree_attn_merge_shards": ([vp, vp, i32, i64, i32, vp, vp, vp], ctypes.c_int),
+            "tree_attn_decode_multi_paged_ex": (
+                [ctypes.c_int, vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, i32, f32, vp, vp, popt, vp, sz,
+                 vp],
+                ctypes.c_int,
+            ),
             "tree_attn_decode_paged": (
                 [vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
@@ -322,3 +328,18 @@ def tree_attn_merge_shards(outs, lses, n_shards, rows, head_dim, out, lse, strea
     """Merge (out, lse) computed over n_shards slices of every sequence: outs [n_shards][rows][D]."""
     _check(lib().tree_attn_merge_shards(_ptr(outs), _ptr(lses), n_shards, rows, head_dim, _ptr(out), _ptr(lse),
                                         _stream(stream, outs, out)), "tree_attn_merge_shards")
+
+
+def tree_attn_decode_multi_paged_ex(dtype, q, k_pages, v_pages, num_pages, page_size, block_table,
+                                    block_table_stride, seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, scale,
+                                    out, lse, opts, workspace, workspace_bytes: Optional[int] = None,
+                                    stream=None) -> None:
+    """Several query tokens per sequence over a paged cache: q, out [B][n][Hq][D]."""
+    arr, n = _lens(seqlens)
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().tree_attn_decode_multi_paged_ex(_DTYPES[dtype], _ptr(q), _ptr(k_pages), _ptr(v_pages), num_pages,
+                                                 page_size, _ptr(block_table), block_table_stride, arr, n, n_queries,
+                                                 n_q_heads, n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse),
+                                                 _opts(opts), _ptr(workspace), workspace_bytes,
+                                                 _stream(stream, q, out)), "tree_attn_decode_multi_paged_ex")

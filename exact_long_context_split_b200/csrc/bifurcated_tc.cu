@@ -6,13 +6,20 @@ namespace ta {
 size_t bif_prefix_smem_bytes() { return sizeof(BifSmem) + 1024; }
 
 cudaError_t bif_prefix_set_smem_limit() {
-  return cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel),
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel<false>),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bif_prefix_smem_bytes()));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(reinterpret_cast<const void*>(&bif_prefix_kernel<true>),
                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bif_prefix_smem_bytes()));
 }
 
 cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensorMap& vmap, const BifParams& p,
                               cudaStream_t st) {
-  bif_prefix_kernel<<<grid, kBifThreads, bif_prefix_smem_bytes(), st>>>(kmap, vmap, p);
+  if (p.mode == 1 && p.block_table != nullptr)
+    bif_prefix_kernel<true><<<grid, kBifThreads, bif_prefix_smem_bytes(), st>>>(kmap, vmap, p);
+  else
+    bif_prefix_kernel<false><<<grid, kBifThreads, bif_prefix_smem_bytes(), st>>>(kmap, vmap, p);
   return cudaGetLastError();
 }
 

@@ -379,6 +379,9 @@ __device__ __forceinline__ bool bif_wait(uint64_t* bar, uint32_t parity, const B
 // The prefix kernel
 // ---------------------------------------------------------------------------------------------
 
+// PAGED: mode 1 over a paged cache (a separate instance: the contiguous kernel carries none of
+// the paged producer's code).
+template <bool PAGED>
 __global__ void __launch_bounds__(kBifThreads, 1)
     bif_prefix_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ BifParams p) {
@@ -451,23 +454,76 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     if (lane == 0) {
       uint64_t pol;
       asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-      auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int t) {
-        const int y = static_cast<int>(kv_row0 + (j0 + t) * kBifKeys);
-        mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
-        tma_load_2d(dst, map, 0, y, full, pol);
-        tma_load_2d(dst + kBifKeys * 128, map, 64, y, full, pol);
-      };
       int tk = 0, tv = 0;
-      // K(t) once every product that read K(t - 3) is done, then V(t) once P V(t - 2) is.
-      for (int t = 0; t < n_t && !*abort; ++t) {
-        if (t >= kBifKStages && !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
-          break;
-        issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages], t);
-        ++tk;
-        if (t >= kBifVStages && !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
-          break;
-        issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages], t);
-        ++tv;
+      if constexpr (!PAGED) {
+        auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int t) {
+          const int y = static_cast<int>(kv_row0 + (j0 + t) * kBifKeys);
+          mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
+          tma_load_2d(dst, map, 0, y, full, pol);
+          tma_load_2d(dst + kBifKeys * 128, map, 64, y, full, pol);
+        };
+        // K(t) once every product that read K(t - 3) is done, then V(t) once P V(t - 2) is.
+        for (int t = 0; t < n_t && !*abort; ++t) {
+          if (t >= kBifKStages && !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
+            break;
+          issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages], t);
+          ++tk;
+          if (t >= kBifVStages && !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
+            break;
+          issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages], t);
+          ++tv;
+        }
+      } else {
+        // A tile is n_sub boxes of bs rows: one box of 128 rows of a contiguous cache, or one per
+        // page segment of a paged one (the 128-byte swizzle repeats every 8 rows, so boxes of 16
+        // or more rows at their row offsets build the same tile layout as one 128-row box).
+        constexpr bool paged = true;
+        const int bs = paged ? min(1 << p.log2_page, kBifKeys) : kBifKeys;
+        const int n_sub = kBifKeys / bs;
+        int y_sub[kBifKeys / 16];
+        // Tensor-map rows of tile t's boxes; false if a block-table entry is outside the pool.
+        auto locate = [&](int t) -> bool {
+          const int64_t t0 = (j0 + t) * kBifKeys;
+          if (!paged) {
+            y_sub[0] = static_cast<int>(kv_row0 + t0);
+            return true;
+          }
+          const int64_t last_blk = (kv_len - 1) >> p.log2_page;
+          bool good = true;
+          for (int k = 0; k < n_sub; ++k) {
+            const int64_t tok = t0 + static_cast<int64_t>(k) * bs;
+            const int64_t blk = tok >> p.log2_page;
+            // Boxes past the sequence's end read its last block (their keys are masked).
+            const int64_t page = __ldg(p.block_table + b * p.bt_stride + min(blk, last_blk));
+            good = good && page >= 0 && page < p.num_pages;
+            const int64_t off = blk > last_blk ? 0 : (tok & ((int64_t(1) << p.log2_page) - 1));
+            y_sub[k] = static_cast<int>(((page * p.n_kv_heads + h) << p.log2_page) + off);
+          }
+          return good;
+        };
+        auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full) {
+          mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
+          for (int k = 0; k < n_sub; ++k) {
+            tma_load_2d(dst + k * bs * 128, map, 0, y_sub[k], full, pol);
+            tma_load_2d(dst + kBifKeys * 128 + k * bs * 128, map, 64, y_sub[k], full, pol);
+          }
+        };
+        // K(t) once every product that read K(t - 3) is done, then V(t) once P V(t - 2) is.
+        for (int t = 0; t < n_t && !*abort; ++t) {
+          if (!locate(t)) {  // entries load before the stage wait; checked before any copy
+            atomicCAS(p.err, 0, kErrBifBadPage);
+            *abort = 1;
+            break;
+          }
+          if (t >= kBifKStages && !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
+            break;
+          issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages]);
+          ++tk;
+          if (t >= kBifVStages && !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
+            break;
+          issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages]);
+          ++tv;
+        }
       }
       // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
       for (int s = 0; s < kBifKStages && s < tk; ++s) {
@@ -549,6 +605,13 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       const int s = i % kBifVStages;
       if (!bif_wait(&sm.v_full[s], (i / kBifVStages) & 1, p, abort)) break;
       uint4* v4 = reinterpret_cast<uint4*>(sm.v[s]);
+      // Rows past the unit's keys hold whatever follows it (another head, a free page): their
+      // scores are masked, but 0 * NaN is NaN in P V, so they are zeroed.
+      const int64_t valid = kv_len - (j0 + i) * static_cast<int64_t>(kBifKeys);
+      if (valid < kBifKeys) {
+        for (int c = ct; c < 2 * kBifKeys * 128 / 16; c += 64)
+          if (((c & 1023) >> 3) >= valid) v4[c] = make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll 4
       for (int c = ct; c < 2 * kBifKeys * 128 / 16; c += 64) {
         uint4 w = v4[c];

@@ -15,6 +15,7 @@ constexpr int kBifKeys = 128;       // keys per tile (N of S, K of P V)
 constexpr int kBifD = 128;          // head_dim
 constexpr int kBifThreads = 384;    // 12 warps
 constexpr int kErrBifWait = 4;
+constexpr int kErrBifBadPage = 8;  // same word value as the split kernel's bad-page code
 constexpr int kBifPartRow = kBifD + 4;  // floats per partial row: m, l, 2 pad, o[D] (16-byte aligned o)
 constexpr int kBifMaxSeq = 128;         // sequences per launch of the several-query-tokens form
 
@@ -40,6 +41,13 @@ struct BifParams {
   int n_queries;
   int64_t kv_row0[kBifMaxSeq];  // mode 1: tensor-map row of key 0 of sequence b, KV head 0
   int64_t kv_len[kBifMaxSeq];   // mode 1: S_b
+  // Mode 1 over a paged cache (block_table != nullptr): the tensor maps cover the page pools
+  // [num_pages][Hkv][page_size][D] with boxes of min(page_size, 128) rows; sequence b's block i
+  // is page block_table[b * bt_stride + i] (the launch group's first sequence's row first).
+  const int32_t* block_table;
+  int64_t bt_stride;
+  int64_t num_pages;
+  int log2_page;
 };
 
 // Dynamic shared memory of bif_prefix_kernel (the tile ring plus 1 KB for 1024-byte alignment).

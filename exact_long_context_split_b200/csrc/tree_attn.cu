@@ -359,7 +359,7 @@ struct MultiPlan {
 };
 
 ta_status bif_tc_setup(int* sms);
-ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows);
+ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows);
 
 ta_status multi_validate(const DecodeArgs& a, int n_queries, const ta_options* opts, bool check_pointers,
                          KernelInfo* ki) {
@@ -371,7 +371,8 @@ ta_status multi_validate(const DecodeArgs& a, int n_queries, const ta_options* o
   return TA_OK;
 }
 
-ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts, MultiPlan* mp_out) {
+ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts, MultiPlan* mp_out,
+                     const PagedCache* pc = nullptr) {
   const int G = a.Hq / a.Hkv;
   MultiPlan& P = *mp_out;
   P = MultiPlan();
@@ -379,6 +380,7 @@ ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts,
   // tensor map's 32-bit coordinates.
   int64_t cache_rows = 0;
   for (int b = 0; b < a.batch; ++b) cache_rows += a.seqlens[b] * a.Hkv;
+  if (pc) cache_rows = (pc->num_pages * a.Hkv) << pc->log2_page;
   const int rows = G * n_queries;
   const bool tc_ok = a.dt == TA_BF16 && a.D == kBifD && rows <= kBifRows && cache_rows < (int64_t(1) << 31) &&
                      a.kv_offsets == nullptr;
@@ -411,7 +413,8 @@ ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts,
     MultiPass mp;
     mp.q_first = j0;
     mp.n_q = nq;
-    if (!pick_kernel(a.dt, a.D, G * nq, short_tiles, &mp.ki)) return TA_ERR_UNSUPPORTED;
+    if (!pick_kernel(a.dt, a.D, G * nq, short_tiles, &mp.ki, pc != nullptr)) return TA_ERR_UNSUPPORTED;
+    if (pc && mp.ki.tile / (1 << pc->log2_page) + 1 > 32) return TA_ERR_UNSUPPORTED;
     int dev = 0, slots = 1;
     if (a.batch > 0) {
       const ta_status s = resident_ctas(mp.ki, &dev, &slots);
@@ -428,24 +431,29 @@ ta_status multi_plan(const DecodeArgs& a, int n_queries, const ta_options* opts,
 }
 
 ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, const MultiPlan& P, void* ws,
-                    size_t ws_bytes, cudaStream_t st) {
+                    size_t ws_bytes, cudaStream_t st, const PagedCache* pc = nullptr) {
   if (!ws || !aligned(ws, kAlign) || ws_bytes < kHeaderBytes + P.body) return TA_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
   int* err = reinterpret_cast<int*>(base);
   if (!P.tc) {
     for (const MultiPass& mp : P.passes) {
       const ta_status s = launch_plan(mp.plan, mp.ki, a.q, a.k, a.v, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, a.dt,
-                                      opts, base + kHeaderBytes, err, st, n_queries, mp.q_first);
+                                      opts, base + kHeaderBytes, err, st, n_queries, mp.q_first, pc);
       if (s != TA_OK) return s;
     }
     return TA_OK;
   }
   int64_t cache_rows = 0;
   for (int b = 0; b < a.batch; ++b) cache_rows += a.seqlens[b] * a.Hkv;
+  int box_rows = kBifKeys;
+  if (pc) {  // the maps cover the page pools; one box per page segment of a key tile
+    cache_rows = (pc->num_pages * a.Hkv) << pc->log2_page;
+    box_rows = std::min(1 << pc->log2_page, kBifKeys);
+  }
   CUtensorMap kmap, vmap;
-  ta_status s = encode_cache_map(&kmap, a.k, cache_rows);
+  ta_status s = encode_cache_map(&kmap, a.k, cache_rows, box_rows);
   if (s != TA_OK) return s;
-  s = encode_cache_map(&vmap, a.v, cache_rows);
+  s = encode_cache_map(&vmap, a.v, cache_rows, box_rows);
   if (s != TA_OK) return s;
   float* part = reinterpret_cast<float*>(base + kHeaderBytes);
   int64_t row0 = 0;  // tensor-map row of the group's first sequence
@@ -472,6 +480,12 @@ ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, 
     bp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
     bp.mode = 1;
     bp.n_queries = n_queries;
+    if (pc) {
+      bp.block_table = pc->table + static_cast<int64_t>(b0) * pc->stride;
+      bp.bt_stride = pc->stride;
+      bp.num_pages = pc->num_pages;
+      bp.log2_page = pc->log2_page;
+    }
     cudaError_t e = launch_bif_prefix(dim3(bp.n_chunks, a.Hkv, nb), kmap, vmap, bp, st);
     if (e != cudaSuccess) return cuda_fail(e);
     e = launch_merge_chunks(part, bp.n_chunks, a.Hkv, P.rows, n_queries, a.out + qrow0 * a.D, a.lse + qrow0, nb,
@@ -584,13 +598,13 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// [rows][128] bf16 matrix, 64 x 64 boxes, 128-byte swizzle.
-bool encode_kv_map(CUtensorMap* map, const void* base, int64_t rows) {
+// [rows][128] bf16 matrix, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows = kBifKeys) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn || rows <= 0 || rows >= (int64_t(1) << 31)) return false;  // tile rows are 32-bit coordinates
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kBifD), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kBifD) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kBifKeys)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -598,9 +612,9 @@ bool encode_kv_map(CUtensorMap* map, const void* base, int64_t rows) {
 }
 
 // The whole packed cache as one [rows][128] bf16 matrix for the tensor-core passes.
-ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows) {
+ta_status encode_cache_map(CUtensorMap* map, const void* base, int64_t rows, int box_rows) {
   if (rows <= 0) rows = 1;  // no key is read; the map only has to be valid
-  return encode_kv_map(map, base, rows) ? TA_OK : TA_ERR_UNSUPPORTED;
+  return encode_kv_map(map, base, rows, box_rows) ? TA_OK : TA_ERR_UNSUPPORTED;
 }
 
 ta_status bif_tc_setup(int* sms) {
@@ -698,6 +712,7 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
     const bool maps = encode_kv_map(&kmap, a.kp, kv_rows) && encode_kv_map(&vmap, a.vp, kv_rows);
     if (maps) {
       BifParams bpp;
+      std::memset(&bpp, 0, sizeof(bpp));  // mode 0, contiguous prefix: no block table
       bpp.q = a.q;
       bpp.part = reinterpret_cast<float*>(base + bp.part_off);
       bpp.err = err;
@@ -944,6 +959,32 @@ ta_status tree_attn_decode_multi(const void* q, const void* k_cache, const void*
   if (s != TA_OK) return s;
   MultiCtx ctx{a, n_queries, &plan};
   return with_temp_workspace(kHeaderBytes + plan.body, static_cast<cudaStream_t>(stream), &multi_alloc_run, &ctx);
+}
+
+ta_status tree_attn_decode_multi_paged_ex(ta_dtype dtype, const void* q, const void* k_pages, const void* v_pages,
+                                          int64_t num_pages, int32_t page_size, const int32_t* block_table,
+                                          int64_t block_table_stride, const int64_t* seqlens, int32_t batch,
+                                          int32_t n_queries, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          float scale, float* out, float* lse, const ta_options* opts,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  DecodeArgs a{dtype, q, k_pages, v_pages, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
+               scale, out, lse};
+  if (page_size < 16 || page_size > 65536 || (page_size & (page_size - 1)) != 0 || num_pages < 0)
+    return TA_ERR_INVALID_ARG;
+  PagedCache pc{block_table, block_table_stride, num_pages, 0};
+  while ((1 << pc.log2_page) < page_size) ++pc.log2_page;
+  KernelInfo ki;
+  ta_status s = multi_validate(a, n_queries, opts, true, &ki);
+  if (s != TA_OK || batch == 0) return s;
+  int64_t max_blocks = 0;
+  for (int b = 0; b < batch; ++b) max_blocks = std::max<int64_t>(max_blocks, (seqlens[b] + page_size - 1) / page_size);
+  if (block_table_stride < max_blocks || num_pages < 1 || !block_table ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3) != 0)
+    return TA_ERR_INVALID_ARG;
+  MultiPlan plan;
+  s = multi_plan(a, n_queries, opts, &plan, &pc);
+  if (s != TA_OK) return s;
+  return multi_run(a, n_queries, opts, plan, workspace, workspace_bytes, static_cast<cudaStream_t>(stream), &pc);
 }
 
 namespace {

@@ -253,6 +253,19 @@ ta_status tree_attn_decode_paged_ex(ta_dtype dtype, const void* q, const void* k
                                     float* lse, const ta_options* opts, void* workspace, size_t workspace_bytes,
                                     void* stream);
 
+/*
+ * Several query tokens per sequence (tree_attn_decode_multi_ex) over a paged cache
+ * (tree_attn_decode_paged_ex): q, out, lse and the query-token rules of the first, pages,
+ * block table and page rules of the second.  Workspace: tree_attn_multi_workspace_size.  The
+ * tensor-core form reads each 128-key tile as one TMA box per page segment it spans.
+ */
+ta_status tree_attn_decode_multi_paged_ex(ta_dtype dtype, const void* q, const void* k_pages, const void* v_pages,
+                                          int64_t num_pages, int32_t page_size, const int32_t* block_table,
+                                          int64_t block_table_stride, const int64_t* seqlens, int32_t batch,
+                                          int32_t n_queries, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                          float scale, float* out, float* lse, const ta_options* opts,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
 /* Paged decode, bf16, allocating its workspace per call like tree_attn_decode. */
 ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, int64_t num_pages,
                                  int32_t page_size, const int32_t* block_table, int64_t block_table_stride,

@@ -22,6 +22,7 @@ from .attention import (  # noqa: F401
     multi_query_attention,
     online_softmax,
     paged_decode_attention,
+    paged_multi_query_attention,
     sequence_block,
     shard_bounds,
     split_attention,

@@ -384,3 +384,17 @@ def merge_shard_results(outs, lses):
     parts = [(float(l), 1.0 if l != -math.inf else 0.0, np.asarray(o, dtype=np.float64) if l != -math.inf
               else np.zeros_like(np.asarray(o, dtype=np.float64))) for o, l in zip(outs, lses)]
     return finalize(merge_tree(parts))
+
+
+def paged_multi_query_attention(q, k_pages, v_pages, block_table, seqlens: Sequence[int], page_size: int,
+                                n_queries: int, n_q_heads: int, n_kv_heads: int, head_dim: int, scale: float,
+                                dtype: str = "bf16", rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Several query tokens per sequence (reading 7) over a paged cache (reading 8): each
+    sequence's cache gathered through its block-table row, then multi_query_attention."""
+    B, Hkv, D = len(seqlens), n_kv_heads, head_dim
+    kc = np.concatenate([gather_paged_sequence(k_pages, block_table[b], seqlens[b], Hkv, page_size, D).reshape(-1)
+                         for b in range(B)])
+    vc = np.concatenate([gather_paged_sequence(v_pages, block_table[b], seqlens[b], Hkv, page_size, D).reshape(-1)
+                         for b in range(B)])
+    return multi_query_attention(q, kc, vc, seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, scale, dtype=dtype,
+                                 rows=rows)

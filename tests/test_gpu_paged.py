@@ -167,3 +167,68 @@ def test_long_1m_paged_sampled():
     ref_out, ref_lse = oracle.decode_attention(inp["q"], inp["k"], inp["v"], sp.seqlens, 32, Hkv, D, sp.scale,
                                                pairs=pairs)
     compare(out, lse, ref_out, ref_lse, pairs=pairs)
+
+
+# Several query tokens per sequence over a paged cache: the tensor-core form (one TMA box per
+# page segment of a 128-key tile) and the split-KV passes (paged instances).
+MULTI_CASES = [
+    ([5, 129, 2049], 4, 16, 4, 16),      # 16 rows, 16-token pages (8 boxes per key tile)
+    ([300, 40, 1000], 2, 32, 8, 64),     # 8 rows, 64-token pages
+    ([700, 4], 4, 8, 2, 256),            # pages larger than a key tile
+    ([3000, 16], 16, 64, 8, 32),         # 128 rows
+]
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("case", MULTI_CASES, ids=["ps16", "ps64", "ps256", "rows128"])
+def test_multi_query_paged_against_oracle(case, path):
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    seqlens, n, Hq, Hkv, ps = case
+    sp = synth.DecodeSpec("mpaged", list(seqlens), Hq, Hkv, 128, seed=60 + ps, n_queries=n)
+    inp = synth.make_decode_inputs(sp)
+    table, n_pages = synth.page_table(sp.seed, seqlens, ps, spare=2)
+    kp = synth.scatter_pages(inp["k"], seqlens, Hkv, 128, ps, table, n_pages, NAN["bf16"])
+    vp = synth.scatter_pages(inp["v"], seqlens, Hkv, 128, ps, table, n_pages, NAN["bf16"])
+    B = sp.batch
+    out = torch.full((B, n, Hq, 128), float("nan"), device="cuda")
+    lse = torch.full((B, n, Hq), float("nan"), device="cuda")
+    opts = ta.make_options(prefix_path=path)
+    ws = new_workspace(ta.tree_attn_multi_workspace_size(list(seqlens), n, Hq, Hkv, 128, "bf16", opts))
+    ta.tree_attn_decode_multi_paged_ex("bf16", device_tensor(inp["q"], "bf16"), device_tensor(kp.reshape(-1), "bf16"),
+                                       device_tensor(vp.reshape(-1), "bf16"), n_pages, ps,
+                                       torch.from_numpy(table).cuda(), table.shape[1], list(seqlens), n, Hq, Hkv,
+                                       128, sp.scale, out, lse, opts, ws)
+    assert ta.tree_attn_check(ws) == ta.TA_OK
+    o, l = out.cpu().numpy(), lse.cpu().numpy()
+    ref_out, ref_lse = oracle.paged_multi_query_attention(inp["q"], kp.reshape(-1), vp.reshape(-1), table, seqlens,
+                                                          ps, n, Hq, Hkv, 128, sp.scale)
+    compare(o.reshape(B * n, Hq, 128), l.reshape(B * n, Hq), ref_out.reshape(B * n, Hq, 128),
+            ref_lse.reshape(B * n, Hq))
+
+
+def test_multi_query_paged_bad_entry():
+    """A bad block-table entry in the tensor-core form: TA_ERR_BAD_PAGE, NaN rows, no read."""
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    seqlens, n, Hq, Hkv, ps = [300, 70], 2, 8, 2, 16
+    sp = synth.DecodeSpec("mpaged_bad", seqlens, Hq, Hkv, 128, seed=61, n_queries=n)
+    inp = synth.make_decode_inputs(sp)
+    table, n_pages = synth.page_table(sp.seed, seqlens, ps)
+    kp = synth.scatter_pages(inp["k"], seqlens, Hkv, 128, ps, table, n_pages, NAN["bf16"])
+    bad = table.copy()
+    bad[0, 3] = n_pages
+    out = torch.empty(2, n, Hq, 128, device="cuda")
+    lse = torch.empty(2, n, Hq, device="cuda")
+    opts = ta.make_options(prefix_path=1)
+    ws = new_workspace(ta.tree_attn_multi_workspace_size(seqlens, n, Hq, Hkv, 128, "bf16", opts))
+    k = device_tensor(kp.reshape(-1), "bf16")
+    ta.tree_attn_decode_multi_paged_ex("bf16", device_tensor(inp["q"], "bf16"), k, k, n_pages, ps,
+                                       torch.from_numpy(bad).cuda(), bad.shape[1], seqlens, n, Hq, Hkv, 128, sp.scale,
+                                       out, lse, opts, ws)
+    assert ta.tree_attn_check(ws) == ta.TA_ERR_BAD_PAGE
+    assert np.isnan(out[0].cpu().numpy()).all()
