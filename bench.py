@@ -378,6 +378,30 @@ class PagedRun(DecodeRun):
                                           stream=stream)
 
 
+class PagedMultiRun(PagedRun):
+    """Several query tokens per sequence over a paged cache (the tensor-core form when eligible)."""
+
+    def __init__(self, spec, torch, ta):
+        super().__init__(spec, torch, ta)
+        B, n, Hq, Hkv, D = spec.batch, spec.n_queries, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+        self.out = torch.empty(B, n, Hq, D, device="cuda")
+        self.lse = torch.empty(B, n, Hq, device="cuda")
+        self.ws = torch.empty(ta.tree_attn_multi_workspace_size(self.seqlens, n, Hq, Hkv, D), dtype=torch.uint8,
+                              device="cuda")
+        ta.tree_attn_workspace_init(self.ws)
+        tc = D == 128 and 8 <= (Hq // Hkv) * n <= 128
+        self.launches_per_step = 2 * ((B + 127) // 128) if tc else self.launches_per_step
+        self.kernel = ("bif_prefix_kernel<paged> + merge_chunks_kernel" if tc else self.kernel) + \
+            " (%d query tokens, %d-token blocks)" % (n, spec.page_size)
+
+    def step(self, stream):
+        sp = self.spec
+        self.ta.tree_attn_decode_multi_paged_ex("bf16", self.dev["q"], self.dev["k"], self.dev["v"], self.num_pages,
+                                                sp.page_size, self.table, self.stride, self.seqlens, sp.n_queries,
+                                                sp.n_q_heads, sp.n_kv_heads, sp.head_dim, sp.scale, self.out,
+                                                self.lse, None, self.ws, stream=stream)
+
+
 class BifurcatedRun:
     """Shared-prefix workload: one call = prefix pass, suffix pass and the exact merge."""
 
@@ -425,6 +449,8 @@ def run_gpu(args, spec) -> None:
 
     if isinstance(spec, synth.BifurcatedSpec):
         run = BifurcatedRun(spec, torch, ta)
+    elif spec.n_queries > 1 and spec.page_size > 0:
+        run = PagedMultiRun(spec, torch, ta)
     elif spec.n_queries > 1:
         run = MultiRun(spec, torch, ta)
     elif spec.page_size > 0:

@@ -282,9 +282,12 @@ def scatter_pages(cache, seqlens: Sequence[int], n_kv_heads: int, head_dim: int,
 
 
 def paged_configs() -> Dict[str, DecodeSpec]:
-    """long_1m's cache in 16-token blocks placed at random (the common serving block size)."""
+    """long_1m's cache, and spec_decode_4's, in 16-token blocks placed at random (the common
+    serving block size)."""
     return {"long_1m_paged": DecodeSpec("long_1m_paged", [1_048_576], 32, 8, 128, seed=3, spike_frac=0.001,
-                                        page_size=16)}
+                                        page_size=16),
+            "spec_decode_4_paged": DecodeSpec("spec_decode_4_paged", [32768] * 8, 32, 8, 128, seed=8, n_queries=4,
+                                              page_size=16)}
 
 
 def make_bifurcated_inputs(spec: BifurcatedSpec) -> Dict[str, np.ndarray]:
