@@ -477,24 +477,34 @@ __global__ void __launch_bounds__(kBifThreads, 1)
         // A tile is n_sub boxes of bs rows: one box of 128 rows of a contiguous cache, or one per
         // page segment of a paged one (the 128-byte swizzle repeats every 8 rows, so boxes of 16
         // or more rows at their row offsets build the same tile layout as one 128-row box).
-        constexpr bool paged = true;
-        const int bs = paged ? min(1 << p.log2_page, kBifKeys) : kBifKeys;
+        const int bs = min(1 << p.log2_page, kBifKeys);
         const int n_sub = kBifKeys / bs;
         int y_sub[kBifKeys / 16];
-        // Tensor-map rows of tile t's boxes; false if a block-table entry is outside the pool.
-        auto locate = [&](int t) -> bool {
+        int32_t pg[kBifKeys / 16];  // block-table entries of the next tile, loaded ahead
+        const int64_t last_blk = (kv_len - 1) >> p.log2_page;
+        // Issue the loads of tile t's entries; their values are used only in resolve(t), after
+        // the stage wait, so the loads' latency overlaps it.  Boxes past the sequence's end
+        // read its last block (their keys are masked and their V rows zeroed).
+        auto fetch = [&](int t) {
           const int64_t t0 = (j0 + t) * kBifKeys;
-          if (!paged) {
-            y_sub[0] = static_cast<int>(kv_row0 + t0);
-            return true;
+#pragma unroll
+          for (int k = 0; k < kBifKeys / 16; ++k) {  // constant indices keep pg[] in registers
+            if (k < n_sub) {
+              const int64_t blk = (t0 + static_cast<int64_t>(k) * bs) >> p.log2_page;
+              pg[k] = __ldg(p.block_table + b * p.bt_stride + min(blk, last_blk));
+            }
           }
-          const int64_t last_blk = (kv_len - 1) >> p.log2_page;
+        };
+        // Tensor-map rows of tile t's boxes; false if an entry is outside the pool.
+        auto resolve = [&](int t) -> bool {
+          const int64_t t0 = (j0 + t) * kBifKeys;
           bool good = true;
-          for (int k = 0; k < n_sub; ++k) {
+#pragma unroll
+          for (int k = 0; k < kBifKeys / 16; ++k) {
+            if (k >= n_sub) break;
             const int64_t tok = t0 + static_cast<int64_t>(k) * bs;
             const int64_t blk = tok >> p.log2_page;
-            // Boxes past the sequence's end read its last block (their keys are masked).
-            const int64_t page = __ldg(p.block_table + b * p.bt_stride + min(blk, last_blk));
+            const int64_t page = pg[k];
             good = good && page >= 0 && page < p.num_pages;
             const int64_t off = blk > last_blk ? 0 : (tok & ((int64_t(1) << p.log2_page) - 1));
             y_sub[k] = static_cast<int>(((page * p.n_kv_heads + h) << p.log2_page) + off);
@@ -503,23 +513,29 @@ __global__ void __launch_bounds__(kBifThreads, 1)
         };
         auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full) {
           mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
-          for (int k = 0; k < n_sub; ++k) {
+#pragma unroll
+          for (int k = 0; k < kBifKeys / 16; ++k) {
+            if (k >= n_sub) break;
             tma_load_2d(dst + k * bs * 128, map, 0, y_sub[k], full, pol);
             tma_load_2d(dst + kBifKeys * 128 + k * bs * 128, map, 64, y_sub[k], full, pol);
           }
         };
+        if (n_t > 0) fetch(0);
         // K(t) once every product that read K(t - 3) is done, then V(t) once P V(t - 2) is.
         for (int t = 0; t < n_t && !*abort; ++t) {
-          if (!locate(t)) {  // entries load before the stage wait; checked before any copy
+          if (t >= kBifKStages &&
+              !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
+            break;
+          if (!resolve(t)) {  // checked before anything is expected on the stage's barrier
             atomicCAS(p.err, 0, kErrBifBadPage);
             *abort = 1;
             break;
           }
-          if (t >= kBifKStages && !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
-            break;
+          if (t + 1 < n_t) fetch(t + 1);
           issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages]);
           ++tk;
-          if (t >= kBifVStages && !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
+          if (t >= kBifVStages &&
+              !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
             break;
           issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages]);
           ++tv;
