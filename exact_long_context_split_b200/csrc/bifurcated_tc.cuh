@@ -450,8 +450,9 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------
     // K and V tiles in order; a K stage refills once every S = Q K^T that reads it is done, a
-    // V stage once every P V that reads it is done.
-    if (lane == 0) {
+    // V stage once every P V that reads it is done.  Contiguous: lane 0 alone.  Paged: the
+    // whole warp, lane k issuing the k-th page segment's boxes.
+    if (PAGED || lane == 0) {
       uint64_t pol;
       asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
       int tk = 0, tv = 0;
@@ -478,77 +479,75 @@ __global__ void __launch_bounds__(kBifThreads, 1)
         // page segment of a paged one (the 128-byte swizzle repeats every 8 rows, so boxes of 16
         // or more rows at their row offsets build the same tile layout as one 128-row box).
         const int bs = min(1 << p.log2_page, kBifKeys);
-        const int n_sub = kBifKeys / bs;
-        int y_sub[kBifKeys / 16];
-        int32_t pg[kBifKeys / 16];  // block-table entries of the next tile, loaded ahead
+        const int n_sub = kBifKeys / bs;  // boxes per half-tile, at most 8 (pages of 16+ tokens)
         const int64_t last_blk = (kv_len - 1) >> p.log2_page;
-        // Issue the loads of tile t's entries; their values are used only in resolve(t), after
-        // the stage wait, so the loads' latency overlaps it.  Boxes past the sequence's end
-        // read its last block (their keys are masked and their V rows zeroed).
+        int32_t pg = 0;  // this lane's block-table entry of the next tile, loaded ahead
+        int y = 0;       // this lane's box row of the current tile
+        // Lane k loads tile t's k-th entry; the value is used only in resolve(t), after the stage
+        // wait, so the load's latency overlaps it.  Boxes past the sequence's end read its last
+        // block (their keys are masked and their V rows zeroed).
         auto fetch = [&](int t) {
-          const int64_t t0 = (j0 + t) * kBifKeys;
-#pragma unroll
-          for (int k = 0; k < kBifKeys / 16; ++k) {  // constant indices keep pg[] in registers
-            if (k < n_sub) {
-              const int64_t blk = (t0 + static_cast<int64_t>(k) * bs) >> p.log2_page;
-              pg[k] = __ldg(p.block_table + b * p.bt_stride + min(blk, last_blk));
-            }
+          if (lane < n_sub) {
+            const int64_t blk = ((j0 + t) * kBifKeys + static_cast<int64_t>(lane) * bs) >> p.log2_page;
+            pg = __ldg(p.block_table + b * p.bt_stride + min(blk, last_blk));
           }
         };
-        // Tensor-map rows of tile t's boxes; false if an entry is outside the pool.
+        // Box rows of tile t; false (for every lane) if any entry is outside the pool.
         auto resolve = [&](int t) -> bool {
-          const int64_t t0 = (j0 + t) * kBifKeys;
           bool good = true;
-#pragma unroll
-          for (int k = 0; k < kBifKeys / 16; ++k) {
-            if (k >= n_sub) break;
-            const int64_t tok = t0 + static_cast<int64_t>(k) * bs;
+          if (lane < n_sub) {
+            const int64_t tok = (j0 + t) * kBifKeys + static_cast<int64_t>(lane) * bs;
             const int64_t blk = tok >> p.log2_page;
-            const int64_t page = pg[k];
-            good = good && page >= 0 && page < p.num_pages;
+            const int64_t page = pg;
+            good = page >= 0 && page < p.num_pages;
             const int64_t off = blk > last_blk ? 0 : (tok & ((int64_t(1) << p.log2_page) - 1));
-            y_sub[k] = static_cast<int>(((page * p.n_kv_heads + h) << p.log2_page) + off);
+            y = static_cast<int>(((page * p.n_kv_heads + h) << p.log2_page) + off);
           }
-          return good;
+          return __all_sync(0xffffffffu, good);
         };
         auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full) {
-          mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
-#pragma unroll
-          for (int k = 0; k < kBifKeys / 16; ++k) {
-            if (k >= n_sub) break;
-            tma_load_2d(dst + k * bs * 128, map, 0, y_sub[k], full, pol);
-            tma_load_2d(dst + kBifKeys * 128 + k * bs * 128, map, 64, y_sub[k], full, pol);
+          if (lane == 0) mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
+          __syncwarp();
+          if (lane < n_sub) {
+            tma_load_2d(dst + lane * bs * 128, map, 0, y, full, pol);
+            tma_load_2d(dst + kBifKeys * 128 + lane * bs * 128, map, 64, y, full, pol);
           }
+        };
+        auto stage_wait = [&](uint64_t* bar, uint32_t parity) -> bool {  // lane 0 waits, all learn
+          bool ok = true;
+          if (lane == 0) ok = bif_wait(bar, parity, p, abort);
+          return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         };
         if (n_t > 0) fetch(0);
         // K(t) once every product that read K(t - 3) is done, then V(t) once P V(t - 2) is.
-        for (int t = 0; t < n_t && !*abort; ++t) {
-          if (t >= kBifKStages &&
-              !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
-            break;
+        for (int t = 0; t < n_t; ++t) {
+          if (__shfl_sync(0xffffffffu, *abort ? 1 : 0, 0) != 0) break;
+          if (t >= kBifKStages && !stage_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1)) break;
           if (!resolve(t)) {  // checked before anything is expected on the stage's barrier
-            atomicCAS(p.err, 0, kErrBifBadPage);
-            *abort = 1;
+            if (lane == 0) {
+              atomicCAS(p.err, 0, kErrBifBadPage);
+              *abort = 1;
+            }
             break;
           }
           if (t + 1 < n_t) fetch(t + 1);
           issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages]);
           ++tk;
-          if (t >= kBifVStages &&
-              !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
-            break;
+          if (t >= kBifVStages && !stage_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1)) break;
           issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages]);
           ++tv;
         }
       }
       // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
-      for (int s = 0; s < kBifKStages && s < tk; ++s) {
-        const int last = (tk - 1 - s) / kBifKStages;
-        if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
-      }
-      for (int s = 0; s < kBifVStages && s < tv; ++s) {
-        const int last = (tv - 1 - s) / kBifVStages;
-        if (!wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+      if (lane == 0) {
+        for (int s = 0; s < kBifKStages && s < tk; ++s) {
+          const int last = (tk - 1 - s) / kBifKStages;
+          if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+        }
+        for (int s = 0; s < kBifVStages && s < tv; ++s) {
+          const int last = (tv - 1 - s) / kBifVStages;
+          if (!wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
+        }
       }
     }
     __syncwarp();
