@@ -119,6 +119,7 @@ class ClockSampler:
         self.err = None
         self._stop = False
         self._thread = None
+        self._first = None  # set once the first sample (or an NVML error) exists
 
     def _handle(self, nv):
         import torch
@@ -144,17 +145,22 @@ class ClockSampler:
             while not self._stop:
                 self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
                                      int(get_reasons(h))))
+                self._first.set()
                 time.sleep(self.period)
             nv.nvmlShutdown()
         except Exception as e:  # NVML missing or refused: report it, never fail the bench
             self.err = f"nvml: {e}"
+            self._first.set()
 
     def __enter__(self):
         import threading
 
+        self._first = threading.Event()
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
-        time.sleep(0.05)
+        # NVML's first initialisation can take longer than a short timed region: start timing
+        # only once the sampler is producing samples (bounded).
+        self._first.wait(timeout=10.0)
         return self
 
     def start(self):
