@@ -7,6 +7,9 @@ passages they follow.
 """
 from .attention import (  # noqa: F401
     Partial,
+    anchor_block_attention,
+    anchor_visible_keys,
+    attention_heads_cache,
     attention_one,
     attention_one_bf16_cache,
     bf16_to_f64,

@@ -24,7 +24,8 @@ Sources (the web pages this method is taken from):
   tokens is split into two GEMMs and stays exact.
 * [StarAttn] Star Attention article (tiaojiaomugou.com, 242533), "Phase 2: query
   encoding and token generation": each host attends over its local cache and the
-  query host combines the softmax statistics into global attention.
+  query host combines the softmax statistics into global attention; "Phase 1: context
+  encoding": the context is cut into blocks, each prefixed with the anchor block.
 
 Readings taken where the pages are silent or garbled (each also listed in the
 design notes):
@@ -56,6 +57,15 @@ design notes):
    token range shard_bounds(S, W, r) of every sequence and computes ordinary decode attention
    over it, i.e. (out_r, lse_r); the results combine exactly as partials (m = lse_r, l = 1,
    o = out_r) merged in a fixed pairwise tree over r.  A shard with no token gives (0, -inf).
+10. Context encoding with anchor blocks ([StarAttn], "Two-phase inference under Star Attention",
+   "Phase 1: context encoding"): the context of S tokens is cut into blocks of block_size
+   tokens (the last one may be shorter); every block except the first is prefixed with the
+   first block (the anchor block) and each host attends over its [anchor ; own block]
+   sequence.  Read here, as the page does not spell it out: attention inside that augmented
+   sequence is the usual causal rule, so the token at position p of block i (i = p //
+   block_size) attends to keys [0, p] when i = 0 and to keys [0, block_size) and
+   [i * block_size, p] when i > 0; the anchor block is the first block, of block_size tokens.
+   Only the non-anchor rows of each host are kept, so every position has exactly one output.
 """
 from __future__ import annotations
 
@@ -123,29 +133,41 @@ def attention_one(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> 
     return out, m + math.log(l)
 
 
+def attention_heads_cache(Q: np.ndarray, Kbits: np.ndarray, Vbits: np.ndarray, scale: float,
+                          dtype: str = "bf16") -> Tuple[np.ndarray, np.ndarray]:
+    """attention_one for several query rows over one long cache kept in its storage format.
+
+    Q: [H][D] float64 (the query heads that read this cache); Kbits, Vbits: [S][D] bf16 bits
+    or float32.  The cache is widened to float64 ROWS_PER_PIECE rows at a time.  For every
+    row h the arithmetic is the definition's: pass 1 forms every score x_t = scale * q_h.k_t
+    (one product K Q^T serves all rows) and their maximum m_h before pass 2 forms
+    l_h = sum_t exp(x_t - m_h) and sum_t exp(x_t - m_h) v_t.  Returns (out [H][D], lse [H]).
+    """
+    Q = np.atleast_2d(np.asarray(Q, dtype=np.float64))
+    S = Kbits.shape[0]
+    H, D = Q.shape
+    if S == 0:
+        return np.zeros((H, D)), np.full(H, -math.inf)
+    x = np.empty((S, H))
+    for r0 in range(0, S, ROWS_PER_PIECE):
+        r1 = min(S, r0 + ROWS_PER_PIECE)
+        x[r0:r1] = scale * (to_f64(Kbits[r0:r1], dtype) @ Q.T)
+    m = np.max(x, axis=0)
+    e = np.exp(x - m)
+    l = np.sum(e, axis=0)
+    acc = np.zeros((H, D))
+    for r0 in range(0, S, ROWS_PER_PIECE):
+        r1 = min(S, r0 + ROWS_PER_PIECE)
+        acc += e[r0:r1].T @ to_f64(Vbits[r0:r1], dtype)
+    return acc / l[:, None], m + np.log(l)
+
+
 def attention_one_bf16_cache(q: np.ndarray, Kbits: np.ndarray, Vbits: np.ndarray, scale: float,
                              dtype: str = "bf16") -> Tuple[np.ndarray, float]:
-    """attention_one for a long cache kept in its storage format ([S][D] bf16 bits or float32).
-
-    The cache is widened to float64 ROWS_PER_PIECE rows at a time; pass 1 still
-    forms every score before pass 2 starts, so the arithmetic is the definition's.
-    """
-    S = Kbits.shape[0]
-    D = q.shape[0]
-    if S == 0:
-        return np.zeros(D), -math.inf
-    x = np.empty(S)
-    for r0 in range(0, S, ROWS_PER_PIECE):
-        r1 = min(S, r0 + ROWS_PER_PIECE)
-        x[r0:r1] = scale * (to_f64(Kbits[r0:r1], dtype) @ q)
-    m = float(np.max(x))
-    e = np.exp(x - m)
-    l = float(np.sum(e))
-    acc = np.zeros(D)
-    for r0 in range(0, S, ROWS_PER_PIECE):
-        r1 = min(S, r0 + ROWS_PER_PIECE)
-        acc += e[r0:r1] @ to_f64(Vbits[r0:r1], dtype)
-    return acc / l, m + math.log(l)
+    """attention_one for one query row over a cache kept in its storage format ([S][D] bf16
+    bits or float32): attention_heads_cache with a single row."""
+    out, lse = attention_heads_cache(np.asarray(q, dtype=np.float64)[None, :], Kbits, Vbits, scale, dtype)
+    return out[0], float(lse[0])
 
 
 def decode_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_q_heads: int, n_kv_heads: int,
@@ -174,8 +196,7 @@ def decode_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_q_heads: int
         Vb = sequence_block(v_cache, seqlens, b, Hkv, D)
         for g in sorted({h // G for (bb, h) in todo if bb == b}):
             heads = [h for (bb, h) in todo if bb == b and h // G == g]
-            for h in heads:
-                out[b, h], lse[b, h] = attention_one_bf16_cache(qf[b, h], Kb[g], Vb[g], scale, dtype)
+            out[b, heads], lse[b, heads] = attention_heads_cache(qf[b, heads], Kb[g], Vb[g], scale, dtype)
     return out, lse
 
 
@@ -336,13 +357,11 @@ def multi_query_attention(q, k_cache, v_cache, seqlens: Sequence[int], n_queries
         Kb = sequence_block(k_cache, seqlens, b, Hkv, D)
         Vb = sequence_block(v_cache, seqlens, b, Hkv, D)
         S = int(seqlens[b])
-        for (bb, j, h) in todo:
-            if bb != b:
-                continue
+        for (j, g) in sorted({(r[1], r[2] // G) for r in todo if r[0] == b}):
+            heads = [h for (bb, jj, h) in todo if bb == b and jj == j and h // G == g]
             visible = S - n + j + 1
-            g = h // G
-            out[b, j, h], lse[b, j, h] = attention_one_bf16_cache(qf[b, j, h], Kb[g][:visible], Vb[g][:visible],
-                                                                  scale, dtype)
+            out[b, j, heads], lse[b, j, heads] = attention_heads_cache(qf[b, j, heads], Kb[g][:visible],
+                                                                       Vb[g][:visible], scale, dtype)
     return out, lse
 
 
@@ -398,3 +417,44 @@ def paged_multi_query_attention(q, k_pages, v_pages, block_table, seqlens: Seque
                          for b in range(B)])
     return multi_query_attention(q, kc, vc, seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, scale, dtype=dtype,
                                  rows=rows)
+
+
+def anchor_visible_keys(position: int, block_size: int) -> np.ndarray:
+    """Key indices the token at `position` attends to in context encoding (reading 10): the
+    anchor block's keys [0, block_size) (for blocks after the first) and its own block's keys up
+    to and including itself."""
+    i = position // block_size
+    own = np.arange(i * block_size, position + 1)
+    if i == 0:
+        return own
+    return np.concatenate([np.arange(block_size), own])
+
+
+def anchor_block_attention(q, k, v, seq_len: int, block_size: int, n_q_heads: int, n_kv_heads: int,
+                           head_dim: int, scale: float, dtype: str = "bf16",
+                           rows: Optional[Iterable[Tuple[int, int]]] = None):
+    """Star Attention phase 1 (context encoding with anchor blocks, reading 10) for one context.
+
+    q: [S][Hq][D] (the S context tokens' queries, storage format); k, v: [Hkv][S][D].  Query
+    head h of position p attends over KV head h // G at the keys anchor_visible_keys(p, B).
+    Returns (out [S][Hq][D], lse [S][Hq]) in float64.  With `rows`, only those (p, h) entries
+    are computed; the rest are NaN.
+    """
+    S, Hq, Hkv, D, B = int(seq_len), n_q_heads, n_kv_heads, head_dim, int(block_size)
+    if Hq % Hkv != 0:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    if B < 1:
+        raise ValueError("block_size must be positive")
+    G = Hq // Hkv
+    qf = to_f64(np.asarray(q).reshape(S, Hq, D), dtype)
+    K = np.asarray(k).reshape(Hkv, S, D)
+    V = np.asarray(v).reshape(Hkv, S, D)
+    out = np.full((S, Hq, D), np.nan)
+    lse = np.full((S, Hq), np.nan)
+    todo = sorted(set(rows)) if rows is not None else [(p, h) for p in range(S) for h in range(Hq)]
+    for p in sorted({r[0] for r in todo}):
+        keys = anchor_visible_keys(p, B)
+        for g in sorted({h // G for (pp, h) in todo if pp == p}):
+            heads = [h for (pp, h) in todo if pp == p and h // G == g]
+            out[p, heads], lse[p, heads] = attention_heads_cache(qf[p, heads], K[g][keys], V[g][keys], scale, dtype)
+    return out, lse

@@ -394,6 +394,14 @@ def pin_long_cache_pieces(O):
         o1, l1 = O.attention_one_bf16_cache(q, Kb, Vb, 0.3, dtype="bf16")
         o2, l2 = O.attention_one(q, O.bf16_to_f64(Kb), O.bf16_to_f64(Vb), 0.3)
         _close(o1, o2, rtol=1e-12, atol=1e-15, what="pieces bf16")
+        # several query rows in one pass: each row is the definition applied to that row alone
+        Q = r.standard_normal((3, D))
+        Q[2] = -2.0 * Q[0]
+        oh, lh = O.attention_heads_cache(Q, Kb, Vb, 0.3, dtype="bf16")
+        for h in range(3):
+            o2, l2 = O.attention_one(Q[h], O.bf16_to_f64(Kb), O.bf16_to_f64(Vb), 0.3)
+            _close(oh[h], o2, rtol=1e-12, atol=1e-15, what=f"pieces bf16 row {h}")
+            _close(lh[h], l2, rtol=1e-14, what=f"pieces bf16 lse row {h}")
     finally:
         mod.ROWS_PER_PIECE = saved
 
@@ -530,6 +538,116 @@ def pin_sharded_decode(O):
         _close(lse, x.max() + math.log(e.sum()), rtol=1e-13, what=f"sharded lse S={S} W={W}")
 
 
+def pin_paged_multi_query(O):
+    """[AttnAccel] part 3 with reading 7: several query tokens over a paged cache.  Contiguous
+    caches are scattered into pages through a random block table with plain numpy fancy
+    indexing (whole pages at once); every row must equal a staircase-masked softmax written
+    here from the contiguous cache (scores of all n query tokens, -inf above the staircase,
+    row softmax).  Two sequences whose tables share their first block read the same rows."""
+    r = _rng(31)
+    D, Hkv, Hq, ps, n = 4, 2, 4, 4, 3
+    seqlens = [9, 3, 14, 5]
+    G, B = Hq // Hkv, len(seqlens)
+    nblk = [-(-S // ps) for S in seqlens]
+    n_pages = sum(nblk) + 2
+    perm = r.permutation(n_pages)
+    table = np.zeros((B, max(nblk)), dtype=np.int64)
+    pk = np.full((n_pages, Hkv, ps, D), np.nan)
+    pv = np.full((n_pages, Hkv, ps, D), np.nan)
+    kb, vb = [], []
+    used = 0
+    for b, S in enumerate(seqlens):
+        kk = r.standard_normal((Hkv, nblk[b] * ps, D))
+        vv = r.standard_normal((Hkv, nblk[b] * ps, D))
+        kk[:, S:] = np.nan  # rows past the sequence never enter the result
+        vv[:, S:] = np.nan
+        kb.append(kk[:, :S])
+        vb.append(vv[:, :S])
+        table[b, :nblk[b]] = perm[used:used + nblk[b]]
+        used += nblk[b]
+        pk[table[b, :nblk[b]]] = kk.reshape(Hkv, nblk[b], ps, D).transpose(1, 0, 2, 3)
+        pv[table[b, :nblk[b]]] = vv.reshape(Hkv, nblk[b], ps, D).transpose(1, 0, 2, 3)
+    q = r.standard_normal((B, n, Hq, D))
+    out, lse = O.paged_multi_query_attention(q, pk.reshape(-1), pv.reshape(-1), table, seqlens, ps, n, Hq, Hkv, D,
+                                             0.8, dtype="f64")
+    for b, S in enumerate(seqlens):
+        hidden = np.triu(np.ones((n, S), dtype=bool), k=S - n + 1)
+        for h in range(Hq):
+            X = 0.8 * (q[b, :, h, :] @ kb[b][h // G].T)
+            X[hidden] = -np.inf
+            mx = X.max(axis=1, keepdims=True)
+            E = np.exp(X - mx)
+            L = E.sum(axis=1)
+            _close(out[b, :, h], (E @ vb[b][h // G]) / L[:, None], rtol=1e-12, atol=1e-14,
+                   what=f"paged multi-query {b},{h}")
+            _close(lse[b, :, h], mx[:, 0] + np.log(L), rtol=1e-13, what=f"paged multi-query lse {b},{h}")
+    # sequence 1 shares sequence 0's first block: its rows are sequence 0's first rows
+    shared = table.copy()
+    shared[1, 0] = table[0, 0]
+    lens = [ps, ps]
+    q2 = np.repeat(q[:1, :1], 2, axis=0)
+    o2, l2 = O.paged_multi_query_attention(q2, pk.reshape(-1), pv.reshape(-1), shared[:2], lens, ps, 1, Hq, Hkv, D,
+                                           0.8, dtype="f64")
+    _close(o2[1], o2[0], rtol=0.0, what="shared first block")
+    _close(l2[1], l2[0], rtol=0.0, what="shared first block lse")
+
+
+def pin_anchor_blocks(O):
+    """[StarAttn] phase 1 (reading 10) as the page describes it: each block after the first is
+    prefixed with the anchor block and the host runs ordinary causal attention over that
+    augmented sequence, keeping the rows of its own block.  Computed here with torch's
+    scaled_dot_product_attention (is_causal) per augmented block; the first block is causal
+    attention over itself.  Also: a block at least as long as the context is plain causal
+    attention, and with identical keys every row is the mean of its visible value rows."""
+    import torch
+
+    r = _rng(33)
+    D, Hkv, Hq = 8, 2, 4
+    G = Hq // Hkv
+    for S, Bsz in ((23, 6), (16, 4), (9, 9), (7, 20)):
+        q = r.standard_normal((S, Hq, D))
+        k = r.standard_normal((Hkv, S, D))
+        v = r.standard_normal((Hkv, S, D))
+        out, lse = O.anchor_block_attention(q, k.reshape(-1), v.reshape(-1), S, Bsz, Hq, Hkv, D, 0.45, dtype="f64")
+        for i0 in range(0, S, Bsz):
+            i1 = min(S, i0 + Bsz)
+            idx = np.arange(i0, i1) if i0 == 0 else np.concatenate([np.arange(min(Bsz, S)), np.arange(i0, i1)])
+            keep = slice(len(idx) - (i1 - i0), len(idx))
+            for h in range(Hq):
+                g = h // G
+                tq = torch.from_numpy(q[idx, h, :]).view(1, 1, len(idx), D)
+                tk = torch.from_numpy(k[g][idx]).view(1, 1, len(idx), D)
+                tv = torch.from_numpy(v[g][idx]).view(1, 1, len(idx), D)
+                ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=0.45)
+                _close(out[i0:i1, h], ref.view(len(idx), D).numpy()[keep], rtol=1e-11, atol=1e-13,
+                       what=f"anchor S={S} B={Bsz} block {i0} head {h}")
+                X = 0.45 * (q[idx, h, :] @ k[g][idx].T)
+                X[np.triu(np.ones((len(idx), len(idx)), dtype=bool), k=1)] = -np.inf
+                import scipy.special
+                _close(lse[i0:i1, h], scipy.special.logsumexp(X, axis=1)[keep], rtol=1e-13,
+                       what=f"anchor lse S={S} B={Bsz} block {i0} head {h}")
+        if Bsz >= S:  # one block: plain causal attention
+            for h in range(Hq):
+                X = 0.45 * (q[:, h, :] @ k[h // G].T)
+                X[np.triu(np.ones((S, S), dtype=bool), k=1)] = -np.inf
+                E = np.exp(X - X.max(axis=1, keepdims=True))
+                _close(out[:, h], (E @ v[h // G]) / E.sum(axis=1, keepdims=True), rtol=1e-12, atol=1e-14,
+                       what="one block is causal attention")
+    # identical keys: out = mean of the visible value rows, lse = s q.k + ln(count)
+    S, Bsz = 13, 4
+    kc = r.standard_normal(D)
+    k = np.tile(kc, (Hkv, S, 1))
+    v = r.standard_normal((Hkv, S, D))
+    q = r.standard_normal((S, Hq, D))
+    out, lse = O.anchor_block_attention(q, k.reshape(-1), v.reshape(-1), S, Bsz, Hq, Hkv, D, 0.3, dtype="f64")
+    for p in range(S):
+        i = p // Bsz
+        vis = list(range(i * Bsz, p + 1)) if i == 0 else list(range(Bsz)) + list(range(i * Bsz, p + 1))
+        for h in range(Hq):
+            _close(out[p, h], v[h // G][vis].mean(axis=0), rtol=1e-12, atol=1e-14, what=f"anchor mean {p},{h}")
+            _close(lse[p, h], 0.3 * float(q[p, h] @ kc) + math.log(len(vis)), rtol=1e-13, what=f"anchor count {p}")
+
+
 ALL_PINS = [
     pin_bf16_decoding,
     pin_identical_keys,
@@ -552,4 +670,6 @@ ALL_PINS = [
     pin_multi_query,
     pin_paged_cache,
     pin_sharded_decode,
+    pin_paged_multi_query,
+    pin_anchor_blocks,
 ]

@@ -40,7 +40,21 @@ MUTANTS = {
     "paged rows ignore the head": ("pages[int(block_row[t // ps]), :, t % ps, :]", "pages[int(block_row[t // ps]), :1, t % ps, :]"),
     "shard bounds overlap": ("    return shard * S // n_shards, (shard + 1) * S // n_shards", "    return shard * S // n_shards, min(S, (shard + 1) * S // n_shards + 1)"),
     "shard merge ignores lse": ("    parts = [(float(l), 1.0 if l != -math.inf", "    parts = [(0.0 if l != -math.inf else l, 1.0 if l != -math.inf"),
-    "pieces skip last rows": ("        acc += e[r0:r1] @ to_f64(Vbits[r0:r1], dtype)", "        acc += e[r0:r1 - (r1 == S)] @ to_f64(Vbits[r0:r1 - (r1 == S)], dtype)"),
+    "pieces skip last rows": ("        acc += e[r0:r1].T @ to_f64(Vbits[r0:r1], dtype)", "        acc += e[r0:r1 - (r1 == S)].T @ to_f64(Vbits[r0:r1 - (r1 == S)], dtype)"),
+    "heads' lse takes the first row's max": ("    return acc / l[:, None], m + np.log(l)", "    return acc / l[:, None], m[0] + np.log(l)"),
+    "heads read each other's scores": ("    x = np.empty((S, H))\n", "    x = np.empty((S, H))\n    Q = Q[::-1]\n"),
+    "paged multi-query reads table row 0": ("kc = np.concatenate([gather_paged_sequence(k_pages, block_table[b],",
+                                            "kc = np.concatenate([gather_paged_sequence(k_pages, block_table[0],"),
+    "paged multi-query V from K pages": ("vc = np.concatenate([gather_paged_sequence(v_pages,", "vc = np.concatenate([gather_paged_sequence(k_pages,"),
+    "paged multi-query cache one row short": ("    return multi_query_attention(q, kc, vc, seqlens, n_queries,",
+                                              "    return multi_query_attention(q, kc, vc, [int(s) - 1 for s in seqlens], n_queries,"),
+    "anchor dropped": ("    if i == 0:\n        return own\n", "    if True:\n        return own\n"),
+    "anchor is the previous block": ("np.concatenate([np.arange(block_size), own])",
+                                     "np.concatenate([np.arange(max(0, i - 1) * block_size, i * block_size), own])"),
+    "own block excludes itself": ("    own = np.arange(i * block_size, position + 1)", "    own = np.arange(i * block_size, position)"),
+    "block index off by one": ("    i = position // block_size\n", "    i = (position + 1) // block_size\n"),
+    "anchor sees the whole own block": ("    own = np.arange(i * block_size, position + 1)",
+                                        "    own = np.arange(i * block_size, (i + 1) * block_size)"),
 }
 
 
