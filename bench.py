@@ -11,11 +11,18 @@ seeded (4.3 GB of K/V, larger than the 126 MB L2, so no flush between steps).
 Prints one JSON line (rank 0).  Under torchrun with N > 1 every rank runs its own
 replica of the workload (no data-path collective: the path does not shard), the
 timed region is bracketed by a barrier and synchronisation, and the time is the max
-over ranks.  `--impl reference` times the CPU oracle on a bounded sample instead.
+over ranks.  `--impl reference` times the CPU oracle instead: every step is a full
+step of the workload (all rows), threaded over (sequence, query head) rows.
+
+Other workloads (--workload): the decode configurations, several query tokens per
+sequence, paged caches, the shared-prefix (bifurcated) step and context encoding with
+anchor blocks.  Each line's roofline is that of the step's main kernel, timed alone with
+CUDA events that the library records around its launches (tree_attn_profile_events).
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import hashlib
 import json
 import os
@@ -33,7 +40,9 @@ import synth  # noqa: E402
 
 METRIC = "decode-attn KV GB/s & % of B200 HBM peak at 1M ctx; µs/step, KV tokens/s"
 UNIT = "GB/s"
+ANCHOR_METRIC = "context-encoding attention TFLOP/s (anchor-block mask, exact); µs/step, tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["exact_long_context_split_b200/csrc/split_kv.cuh", "exact_long_context_split_b200/csrc/ptx.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kv_traffic.json")
 
@@ -76,13 +85,15 @@ def kernel_hash() -> str:
 
 
 def measured_peaks():
+    """(HBM GB/s, dense bf16 TF/s burst, kind): the measured copy and GEMM peaks of this
+    pool's B200s, else the recorded fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as fh:
             d = json.load(fh)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def traffic_per_launch(spec) -> object:
@@ -103,10 +114,19 @@ def traffic_per_launch(spec) -> object:
     return int(round(rd + wr))
 
 
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons read through NVML every 2 ms by a host
-    thread while the timed region runs (a step here lasts under a millisecond, far below
-    nvidia-smi's 200 ms sampling).  Only reads device state."""
+    """SM clock and clock-event (throttle) reasons read through NVML while the timed region
+    runs: a host thread samples every 2 ms, and start() and stop() each take one sample
+    themselves, so the window always holds its two edge samples even when it is shorter than
+    the sampling period.  Only reads device state."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown"}
@@ -117,9 +137,11 @@ class ClockSampler:
         self.samples = []
         self.window = [None, None]
         self.err = None
+        self.max_mhz = None
         self._stop = False
         self._thread = None
-        self._first = None  # set once the first sample (or an NVML error) exists
+        self._nv = None
+        self._h = None
 
     def _handle(self, nv):
         import torch
@@ -131,64 +153,92 @@ class ClockSampler:
         except Exception:
             return nv.nvmlDeviceGetHandleByIndex(self.idx)
 
+    def _sample(self):
+        nv, h = self._nv, self._h
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), int(get_reasons(h))))
+
     def _run(self):
-        import threading  # noqa: F401
-
         try:
-            import pynvml as nv
-
-            nv.nvmlInit()
-            h = self._handle(nv)
-            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                nv.nvmlDeviceGetCurrentClocksThrottleReasons
             while not self._stop:
-                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
-                                     int(get_reasons(h))))
-                self._first.set()
+                self._sample()
                 time.sleep(self.period)
-            nv.nvmlShutdown()
-        except Exception as e:  # NVML missing or refused: report it, never fail the bench
+        except Exception as e:  # never fail the bench on a sampling error
             self.err = f"nvml: {e}"
-            self._first.set()
 
     def __enter__(self):
         import threading
 
-        self._first = threading.Event()
-        self._thread = threading.Thread(target=self._run, daemon=True)
-        self._thread.start()
-        # NVML's first initialisation can take longer than a short timed region: start timing
-        # only once the sampler is producing samples (bounded).
-        self._first.wait(timeout=10.0)
+        try:  # initialised here, before any timing, so the first sample cannot arrive late
+            import pynvml as nv
+
+            nv.nvmlInit()
+            self._nv, self._h = nv, self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:
+            self.err = f"nvml: {e}"
         return self
 
     def start(self):
+        if self._nv is not None and self.err is None:
+            self._sample()
         self.window[0] = time.perf_counter()
 
     def stop(self):
         self.window[1] = time.perf_counter()
+        if self._nv is not None and self.err is None:
+            self._sample()
 
     def __exit__(self, *exc):
         self._stop = True
         if self._thread is not None:
             self._thread.join(timeout=5)
+        if self._nv is not None:
+            try:
+                self._nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
         if self.err or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"], "samples": 0}
         t0, t1 = self.window
-        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1] or self.samples
+        # the edge samples taken by start() and stop() sit just outside [t0, t1]: widen by 1 ms
+        inside = [s for s in self.samples if t0 is not None and t1 is not None and t0 - 1e-3 <= s[0] <= t1 + 1e-3]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples in the timed window"],
+                    "samples": 0}
         reasons = sorted({name for _, _, r in inside for bit, name in self.REASONS.items() if r & bit})
         return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(inside), "source": "nvml, 2 ms"}
+                "samples": len(inside), "source": "nvml: 2 ms thread + start/stop edges"}
 
 
-def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra) -> dict:
+def workload_config(spec, n_gpus: int) -> dict:
+    if isinstance(spec, synth.DecodeSpec):
+        shape = {"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
+                 "query_tokens": spec.n_queries, **({"page_size": spec.page_size} if spec.page_size else {})}
+    elif isinstance(spec, synth.BifurcatedSpec):
+        shape = {"samples": spec.n_samples, "prefix_len": spec.prefix_len,
+                 "suffix_len": int(max(spec.suffix_lens)) if spec.suffix_lens else 0}
+    else:
+        shape = {"seq_len": spec.seq_len, "block_size": spec.block_size}
+    l2 = ("no flush: each step reads %.2f GB of K/V, more than the 126 MB L2" % (spec.kv_bytes / 1e9)
+          if spec.kv_bytes > 2 * 126e6 else
+          "L2 flushed before every step (a 512 MB write outside the timed span)")
+    return {"workload": spec.name, **shape, "n_q_heads": spec.n_q_heads, "n_kv_heads": spec.n_kv_heads,
+            "head_dim": spec.head_dim, "kv_bytes_per_step": spec.kv_bytes, "parallelism": f"replicas{n_gpus}",
+            "l2": l2}
+
+
+def make_record(*, metric, unit, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra) -> dict:
     rec = {
-        "metric": METRIC,
+        "metric": metric,
         "value": value,
-        "unit": UNIT,
+        "unit": unit,
         "n_gpus": n_gpus,
         "steps": steps,
         "warmup": warmup,
@@ -198,54 +248,66 @@ def make_record(*, value, n_gpus, steps, warmup, ms_per_step, spec, dtype, extra
         "vs_baseline": None,
         "dtype": dtype,
         "data": "synthetic",
-        "config": {
-            "workload": spec.name,
-            **({"batch": spec.batch, "seq_len": int(max(spec.seqlens)) if spec.seqlens else 0,
-                "query_tokens": spec.n_queries, **({"page_size": spec.page_size} if spec.page_size else {})}
-               if isinstance(spec, synth.DecodeSpec) else
-               {"samples": spec.n_samples, "prefix_len": spec.prefix_len,
-                "suffix_len": int(max(spec.suffix_lens)) if spec.suffix_lens else 0}),
-            "n_q_heads": spec.n_q_heads,
-            "n_kv_heads": spec.n_kv_heads,
-            "head_dim": spec.head_dim,
-            "kv_bytes_per_step": spec.kv_bytes,
-            "parallelism": f"replicas{n_gpus}",
-            "l2": "no flush: each step reads %.2f GB of K/V, more than the 126 MB L2" % (spec.kv_bytes / 1e9),
-        },
+        "config": workload_config(spec, n_gpus),
     }
     rec.update(extra)
     return rec
 
 
-def oracle_sample_seconds(spec, h_kv: int, q_heads, n_tokens: int = 0) -> float:
-    """Time the CPU oracle on the given query heads of KV head h_kv of sequence 0, over its first
-    n_tokens tokens (0 = all).  Inputs are generated for that head only (the same bytes as the
-    full workload's); only the oracle is timed."""
+# ----------------------------------------------------------------------------------------------
+# The CPU oracle, threaded over (sequence, query head) rows
+# ----------------------------------------------------------------------------------------------
+
+
+def oracle_step_seconds(spec, inp, rows, threads: int) -> float:
+    """Wall time of the CPU oracle computing the given (sequence, query head) rows of a decode
+    workload, one row per task on `threads` threads (numpy releases the GIL in the oracle's array
+    work; BLAS held to one thread per task).  The oracle is called as it stands; only its
+    widening piece size, a memory setting, is lowered so that every thread's pieces fit."""
+    import threadpoolctl
+
     import oracle
+    from oracle import attention as oracle_attention
 
-    S, D, Hq = spec.seqlens[0], spec.head_dim, spec.n_q_heads
-    n = S * D
-    k = synth.normal_bf16(spec.seed, synth.TID_K, n, start=h_kv * n)
-    v = synth.normal_bf16(spec.seed, synth.TID_V, n, start=h_kv * n)
-    if spec.spike_frac > 0:
-        synth.spike_rows_bf16(k.reshape(S, D), spec.seed, h_kv, spec.n_spikes(S), spec.spike_factor)
-    q = synth.normal_bf16(spec.seed, synth.TID_Q, Hq * D).reshape(Hq, D)
-    T = n_tokens or S
-    K, V = k.reshape(S, D)[:T], v.reshape(S, D)[:T]
-    t0 = time.perf_counter()
-    for h in q_heads:
-        oracle.attention_one_bf16_cache(oracle.bf16_to_f64(q[h]), K, V, spec.scale)
-    return time.perf_counter() - t0
+    def one(row):
+        oracle.decode_attention(inp["q"], inp["k"], inp["v"], spec.seqlens, spec.n_q_heads, spec.n_kv_heads,
+                                spec.head_dim, spec.scale, dtype=spec.dtype, pairs=[row])
 
-
-def blas_threads() -> int:
+    saved = oracle_attention.ROWS_PER_PIECE
+    oracle_attention.ROWS_PER_PIECE = 1 << 18
     try:
-        import threadpoolctl
+        with threadpoolctl.threadpool_limits(1), cf.ThreadPoolExecutor(threads) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(one, rows))
+            return time.perf_counter() - t0
+    finally:
+        oracle_attention.ROWS_PER_PIECE = saved
 
-        info = threadpoolctl.threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] or [1])
-    except Exception:
-        return 1
+
+def decode_rows(spec):
+    return [(b, h) for b in range(spec.batch) for h in range(spec.n_q_heads)]
+
+
+def cpu_baseline(spec, inp, budget_s: float = 30.0) -> dict:
+    """The oracle on one full decode step (every row) when a probe says it fits in `budget_s`,
+    else on a bounded sample of rows scaled to the step; threads = min(cores, rows)."""
+    rows = decode_rows(spec)
+    cores = host_cores()
+    threads = max(1, min(cores, len(rows)))
+    probe = oracle_step_seconds(spec, inp, rows[:threads], threads)  # one row per thread
+    est = probe * len(rows) / threads
+    if est <= budget_s:
+        sec = oracle_step_seconds(spec, inp, rows, threads)
+        sample = f"one full step: all {len(rows)} (sequence, query head) rows, {threads} threads"
+    else:
+        n = max(threads, int(len(rows) * budget_s / est) // threads * threads)
+        stride = max(1, len(rows) // n)
+        sub = rows[::stride][:n]
+        sec = oracle_step_seconds(spec, inp, sub, threads) * len(rows) / len(sub)
+        sample = (f"{len(sub)} of {len(rows)} (sequence, query head) rows (every {stride}th), {threads} threads; "
+                  f"step time = sample time x {len(rows)}/{len(sub)}")
+    return {"value": spec.kv_bytes / sec / 1e9, "unit": UNIT, "cores": threads, "host_cores": cores,
+            "kind": "oracle", "sample": sample, "step_s": sec}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -253,29 +315,36 @@ def blas_threads() -> int:
 # ----------------------------------------------------------------------------------------------
 
 
-REF_SLICE = 8  # the reference arm's per-step sample covers 1/REF_SLICE of the sequence
-
-
 def run_reference(args, spec) -> None:
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    G = spec.n_q_heads // spec.n_kv_heads
-    rows = spec.batch * spec.n_q_heads
-    T = spec.seqlens[0] // REF_SLICE
-    for _ in range(args.warmup):
-        oracle_sample_seconds(spec, 0, [0], T)
-    times = [oracle_sample_seconds(spec, i % spec.n_kv_heads, [(i % spec.n_kv_heads) * G], T) for i in range(args.steps)]
-    step_s = statistics.mean(times) * REF_SLICE * rows
+    inp = synth.make_decode_inputs(spec)
+    rows = decode_rows(spec)
+    cores = host_cores()
+    threads = max(1, min(cores, len(rows)))
+    t_first = oracle_step_seconds(spec, inp, rows, threads)  # the first warm-up step, full
+    budget = 180.0  # the whole run stays within a few minutes
+    full = t_first * (args.warmup + args.steps) <= budget
+    if full:
+        sub = rows
+        sample = f"each step: all {len(rows)} (sequence, query head) rows of the workload, {threads} threads"
+    else:
+        n = max(threads, int(len(rows) * budget / (t_first * (args.warmup + args.steps))) // threads * threads)
+        stride = max(1, len(rows) // n)
+        sub = rows[::stride][:n]
+        sample = (f"each step: {len(sub)} of {len(rows)} rows (every {stride}th), {threads} threads; "
+                  f"step time = sample time x {len(rows)}/{len(sub)}")
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_step_seconds(spec, inp, sub, threads)
+    times = [oracle_step_seconds(spec, inp, sub, threads) * len(rows) / len(sub) for _ in range(args.steps)]
+    step_s = statistics.mean(times)
     value = spec.kv_bytes / step_s / 1e9
-    cores = blas_threads()
-    sample = (f"each step: one (sequence, query head) row over the first {T} of {spec.seqlens[0]} tokens "
-              f"(KV head cycling 0..{spec.n_kv_heads - 1}); step time = mean sample time x {REF_SLICE} x {rows} rows")
-    rec = make_record(value=value, n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
-                      spec=spec, dtype="f64", extra={
+    rec = make_record(metric=METRIC, unit=UNIT, value=value, n_gpus=world, steps=args.steps, warmup=args.warmup,
+                      ms_per_step=step_s * 1e3, spec=spec, dtype="f64", extra={
                           "impl": "reference",
-                          "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                           "sample": sample},
+                          "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "host_cores": cores,
+                                           "kind": "oracle", "sample": sample},
                           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
                           "gpu_launches": 0,
                       })
@@ -287,18 +356,23 @@ def run_reference(args, spec) -> None:
 # ----------------------------------------------------------------------------------------------
 
 
+def to_device_bf16(torch, arr):
+    return torch.from_numpy(np.ascontiguousarray(arr).reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
 class DecodeRun:
     """Device and pinned-host buffers of one decode workload and its step (one kernel launch)."""
 
     launches_per_step = 1
+    metric, unit, bound = METRIC, UNIT, "hbm"
 
-    def __init__(self, spec, torch, ta):
+    def __init__(self, spec, torch, ta, keep_inputs=False):
         self.spec, self.torch, self.ta = spec, torch, ta
         B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
         self.seqlens = [int(s) for s in spec.seqlens]
         inp = synth.make_decode_inputs(spec)
-        self.host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
-                     for n in ("q", "k", "v")}
+        self.host = {n: to_device_bf16(torch, inp[n]) for n in ("q", "k", "v")}
+        self.inputs = inp if keep_inputs else None
         del inp
         self.dev = {n: t.cuda() for n, t in self.host.items()}
         self.out = torch.empty(B, Hq, D, device="cuda")
@@ -307,6 +381,7 @@ class DecodeRun:
         ta.tree_attn_workspace_init(self.ws)
         self.kv_bytes = spec.kv_bytes
         self.tokens = spec.tokens
+        self.flops = 4 * D * Hq * sum(self.seqlens)
         self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv},{'ShortTiles' if sum(self.seqlens) < 1024 * len(self.seqlens) else 'LongTiles'}>"
 
     def step(self, stream):
@@ -316,25 +391,30 @@ class DecodeRun:
                                     stream=stream)
 
 
+def multi_visible_keys(seqlens, n):
+    return sum(n * S - n * (n - 1) // 2 for S in seqlens)
+
+
 class MultiRun(DecodeRun):
     """Several query tokens per sequence: one call = the tensor-core form (bf16, D = 128,
     8 <= G n <= 128) or ceil(n G / 8) split-KV passes."""
 
-    def __init__(self, spec, torch, ta):
-        super().__init__(spec, torch, ta)
+    def __init__(self, spec, torch, ta, keep_inputs=False):
+        super().__init__(spec, torch, ta, keep_inputs)
         B, n, Hq, Hkv, D = spec.batch, spec.n_queries, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
         self.out = torch.empty(B, n, Hq, D, device="cuda")
         self.lse = torch.empty(B, n, Hq, device="cuda")
         self.ws = torch.empty(ta.tree_attn_multi_workspace_size(self.seqlens, n, Hq, Hkv, D), dtype=torch.uint8,
                               device="cuda")
         ta.tree_attn_workspace_init(self.ws)
+        self.flops = 4 * D * Hq * multi_visible_keys(self.seqlens, n)
         G = Hq // Hkv
         if D == 128 and 8 <= G * n <= 128:
             # tensor-core form (the library's automatic choice for bf16): per group of up to 128
             # sequences one bif_prefix_kernel launch and one merge_chunks_kernel launch
             groups = (B + 127) // 128
             self.launches_per_step = 2 * groups
-            self.kernel = f"bif_prefix_kernel (several query tokens, {G * n} rows per KV head) + merge_chunks_kernel"
+            self.kernel = f"bif_prefix_kernel (several query tokens, {G * n} rows per KV head)"
         else:
             passes, j = 0, 0
             while j < n:
@@ -357,8 +437,8 @@ class PagedRun(DecodeRun):
     """A paged cache: the contiguous cache laid out in page_size-token blocks at seeded random
     places (built once on the device); each step reads it through the block table."""
 
-    def __init__(self, spec, torch, ta):
-        super().__init__(spec, torch, ta)
+    def __init__(self, spec, torch, ta, keep_inputs=False):
+        super().__init__(spec, torch, ta, keep_inputs)
         Hkv, D, ps = spec.n_kv_heads, spec.head_dim, spec.page_size
         table, self.num_pages = synth.page_table(spec.seed, spec.seqlens, ps)
         self.table = torch.from_numpy(table).cuda()
@@ -387,17 +467,18 @@ class PagedRun(DecodeRun):
 class PagedMultiRun(PagedRun):
     """Several query tokens per sequence over a paged cache (the tensor-core form when eligible)."""
 
-    def __init__(self, spec, torch, ta):
-        super().__init__(spec, torch, ta)
+    def __init__(self, spec, torch, ta, keep_inputs=False):
+        super().__init__(spec, torch, ta, keep_inputs)
         B, n, Hq, Hkv, D = spec.batch, spec.n_queries, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
         self.out = torch.empty(B, n, Hq, D, device="cuda")
         self.lse = torch.empty(B, n, Hq, device="cuda")
         self.ws = torch.empty(ta.tree_attn_multi_workspace_size(self.seqlens, n, Hq, Hkv, D), dtype=torch.uint8,
                               device="cuda")
         ta.tree_attn_workspace_init(self.ws)
+        self.flops = 4 * D * Hq * multi_visible_keys(self.seqlens, n)
         tc = D == 128 and 8 <= (Hq // Hkv) * n <= 128
         self.launches_per_step = 2 * ((B + 127) // 128) if tc else self.launches_per_step
-        self.kernel = ("bif_prefix_kernel<paged> + merge_chunks_kernel" if tc else self.kernel) + \
+        self.kernel = ("bif_prefix_kernel<paged>" if tc else self.kernel) + \
             " (%d query tokens, %d-token blocks)" % (n, spec.page_size)
 
     def step(self, stream):
@@ -409,18 +490,20 @@ class PagedMultiRun(PagedRun):
 
 
 class BifurcatedRun:
-    """Shared-prefix workload: one call = prefix pass, suffix pass and the exact merge."""
+    """Shared-prefix workload: one call = the tensor-core prefix pass, the suffix pass and the
+    exact merge.  The roofline is the prefix pass's dense contraction on the tensor cores."""
 
     launches_per_step = 3
+    metric, unit, bound = METRIC, UNIT, "tensor"
+    inputs = None
 
-    def __init__(self, spec, torch, ta):
+    def __init__(self, spec, torch, ta, keep_inputs=False):
         self.spec, self.torch, self.ta = spec, torch, ta
         N, Hq, Hkv, D = spec.n_samples, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
         self.lens = [int(s) for s in spec.suffix_lens]
         inp = synth.make_bifurcated_inputs(spec)
         names = ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix")
-        self.host = {n: torch.from_numpy(inp[n].reshape(-1).view(np.int16)).view(torch.bfloat16).pin_memory()
-                     for n in names}
+        self.host = {n: to_device_bf16(torch, inp[n]) for n in names}
         del inp
         self.dev = {n: t.cuda() for n, t in self.host.items()}
         self.out = torch.empty(N, Hq, D, device="cuda")
@@ -430,13 +513,57 @@ class BifurcatedRun:
         ta.tree_attn_workspace_init(self.ws)
         self.kv_bytes = spec.kv_bytes
         self.tokens = spec.prefix_len + sum(self.lens)
-        self.kernel = "bifurcated step (prefix pass + suffix pass + merge)"
+        self.flops = 4 * D * N * Hq * spec.prefix_len  # the prefix pass: S = Q K^T and O = P V
+        self.kernel = "bif_prefix_kernel (shared-prefix pass; the step adds the suffix pass and the merge)"
 
     def step(self, stream):
         sp, d = self.spec, self.dev
         self.ta.tree_attn_decode_bifurcated_ex(d["q"], d["k_prefix"], d["v_prefix"], sp.prefix_len, d["k_suffix"],
                                                d["v_suffix"], self.lens, sp.n_q_heads, sp.n_kv_heads, sp.head_dim,
                                                sp.scale, self.out, self.lse, None, self.ws, stream=stream)
+
+
+class AnchorRun:
+    """Context encoding with anchor blocks: one tensor-core launch per step."""
+
+    launches_per_step = 1
+    metric, unit, bound = ANCHOR_METRIC, "TFLOP/s", "tensor"
+    inputs = None
+
+    def __init__(self, spec, torch, ta, keep_inputs=False):
+        self.spec, self.torch, self.ta = spec, torch, ta
+        S, Hq, Hkv, D = spec.seq_len, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+        inp = synth.make_anchor_inputs(spec)
+        self.host = {n: to_device_bf16(torch, inp[n]) for n in ("q", "k", "v")}
+        del inp
+        self.dev = {n: t.cuda() for n, t in self.host.items()}
+        self.out = torch.empty(S, Hq, D, device="cuda")
+        self.lse = torch.empty(S, Hq, device="cuda")
+        self.ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        self.kv_bytes = spec.kv_bytes
+        self.tokens = S
+        self.flops = spec.flops
+        self.kernel = f"bif_prefix_kernel (context encoding, {128 // (Hq // Hkv)} positions x {Hq // Hkv} heads per tile)"
+
+    def step(self, stream):
+        sp, d = self.spec, self.dev
+        self.ta.tree_attn_anchor_prefill(d["q"], d["k"], d["v"], sp.seq_len, sp.block_size, sp.n_q_heads,
+                                         sp.n_kv_heads, sp.head_dim, sp.scale, self.out, self.lse, None, self.ws,
+                                         stream=stream)
+
+
+def make_run(spec, torch, ta, keep_inputs=False):
+    if isinstance(spec, synth.BifurcatedSpec):
+        return BifurcatedRun(spec, torch, ta)
+    if isinstance(spec, synth.AnchorSpec):
+        return AnchorRun(spec, torch, ta)
+    if spec.n_queries > 1 and spec.page_size > 0:
+        return PagedMultiRun(spec, torch, ta, keep_inputs)
+    if spec.n_queries > 1:
+        return MultiRun(spec, torch, ta, keep_inputs)
+    if spec.page_size > 0:
+        return PagedRun(spec, torch, ta, keep_inputs)
+    return DecodeRun(spec, torch, ta, keep_inputs)
 
 
 def run_gpu(args, spec) -> None:
@@ -453,47 +580,53 @@ def run_gpu(args, spec) -> None:
                                 device_id=torch.device("cuda", local_rank))
     import exact_long_context_split_b200 as ta
 
-    if isinstance(spec, synth.BifurcatedSpec):
-        run = BifurcatedRun(spec, torch, ta)
-    elif spec.n_queries > 1 and spec.page_size > 0:
-        run = PagedMultiRun(spec, torch, ta)
-    elif spec.n_queries > 1:
-        run = MultiRun(spec, torch, ta)
-    elif spec.page_size > 0:
-        run = PagedRun(spec, torch, ta)
-    else:
-        run = DecodeRun(spec, torch, ta)
+    want_cpu = world == 1 and not args.no_cpu_baseline and isinstance(spec, synth.DecodeSpec) and \
+        spec.n_queries == 1 and spec.page_size == 0
+    run = make_run(spec, torch, ta, keep_inputs=want_cpu)
     stream = torch.cuda.current_stream()
+    small = spec.kv_bytes <= 2 * 126e6
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda") if small else None
 
     for _ in range(args.warmup):
         run.step(stream)
     torch.cuda.synchronize()
     assert ta.tree_attn_check(run.ws) == ta.TA_OK
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    t_begin = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
+    def events(n):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in ev:  # torch creates the CUDA event on its first record
+            e.record(stream)
+        return ev
+
+    starts, ends = events(args.steps), events(args.steps)
+    kstarts, kends = events(args.steps), events(args.steps)
+    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
         barrier(world)
         torch.cuda.synchronize()
         clocks.start()
-        t_begin.record(stream)
         for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)  # L2 flush outside the step's events
+            ta.tree_attn_profile_events(kstarts[i], kends[i])
             starts[i].record(stream)
             run.step(stream)
             ends[i].record(stream)
-        t_end.record(stream)
+        ta.tree_attn_profile_events()
         torch.cuda.synchronize()
         clocks.stop()
         barrier(world)
     status = ta.tree_attn_check(run.ws)
     if status != ta.TA_OK:
         raise RuntimeError(ta.tree_attn_status_string(status))
-    elapsed_ms = max_over_ranks(t_begin.elapsed_time(t_end), world)
-    kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
-    ms_per_step = elapsed_ms / args.steps
-    value = world * run.kv_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(kstarts, kends))
+    ms_per_step = max_over_ranks(statistics.mean(step_ms), world)
+    elapsed_s = ms_per_step * 1e-3 * args.steps
+    if run.unit == "TFLOP/s":
+        value = world * run.flops / (ms_per_step * 1e-3) / 1e12
+    else:
+        value = world * run.kv_bytes / (ms_per_step * 1e-3) / 1e9
 
     # End to end through the public API: pinned host -> device copies of every input, the
     # call, and the device -> host read of out and lse, every step.
@@ -517,35 +650,38 @@ def run_gpu(args, spec) -> None:
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in run.host.values())
     d2h = out_h.numel() * 4 + lse_h.numel() * 4
+    e2e_value = world * (run.flops / 1e12 if run.unit == "TFLOP/s" else run.kv_bytes / 1e9) / (e2e_ms * 1e-3)
 
-    peak, peak_kind = measured_peaks()
-    achieved = run.kv_bytes / (kernel_ms * 1e-3) / 1e9
+    hbm, bf16, peak_kind = measured_peaks()
+    if run.bound == "tensor":
+        achieved = run.flops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s", "frac": achieved / bf16,
+                "peak_kind": peak_kind + " dense bf16 (burst)", "flops_per_launch": run.flops}
+    else:
+        achieved = run.kv_bytes / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_kind": peak_kind + " copy bandwidth", "bytes_per_launch": run.kv_bytes}
+    roof.update({"kernel": run.kernel, "kernel_us": kernel_ms * 1e3,
+                 "traffic": traffic_per_launch(spec) if type(run) is DecodeRun else None})
     extra = {
-        "ms_per_step": ms_per_step,
         "us_per_step": ms_per_step * 1e3,
-        "kv_tokens_per_s": world * run.tokens * args.steps / (elapsed_ms * 1e-3),
-        "hbm_frac_of_" + peak_kind: value / world / peak,
-        "e2e": {"value": world * run.kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "kv_tokens_per_s": world * run.tokens * args.steps / elapsed_s,
+        "hbm_frac_of_" + peak_kind: world * run.kv_bytes / (ms_per_step * 1e-3) / 1e9 / world / hbm,
+        "e2e": {"value": e2e_value, "unit": run.unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * run.launches_per_step,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_kind": peak_kind, "kernel": run.kernel,
-                     "traffic": traffic_per_launch(spec) if type(run) is DecodeRun else None},
+        "roofline": roof,
         "clocks": clocks.summary(),
+        "build_id": ta.tree_attn_build_id(),
     }
+    if isinstance(run, (BifurcatedRun, AnchorRun)):
+        extra["step_tflops"] = run.flops / (ms_per_step * 1e-3) / 1e12
     if isinstance(run, BifurcatedRun):
         extra["logical_kv_tokens_per_s"] = world * spec.n_samples * (spec.prefix_len + statistics.mean(run.lens)) * \
-            args.steps / (elapsed_ms * 1e-3)
-    if world == 1 and not args.no_cpu_baseline and type(run) is DecodeRun:
-        G = spec.n_q_heads // spec.n_kv_heads
-        sec = oracle_sample_seconds(spec, 0, list(range(G)))
-        rows = spec.batch * spec.n_q_heads
-        cpu_val = spec.kv_bytes / (sec / G * rows) / 1e9
-        extra["cpu_baseline"] = {"value": cpu_val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                                 "sample": f"the {G} query heads of KV head 0 over all {spec.seqlens[0]} tokens took "
-                                           f"{sec:.2f} s; step time = that / {G} x {rows} rows"}
-    rec = make_record(value=value, n_gpus=world, steps=args.steps, warmup=args.warmup, ms_per_step=ms_per_step,
-                      spec=spec, dtype="bf16", extra=extra)
+            args.steps / elapsed_s
+    if want_cpu:
+        extra["cpu_baseline"] = cpu_baseline(spec, run.inputs)
+    rec = make_record(metric=run.metric, unit=run.unit, value=value, n_gpus=world, steps=args.steps,
+                      warmup=args.warmup, ms_per_step=ms_per_step, spec=spec, dtype="bf16", extra=extra)
     if rank == 0:
         print(json.dumps(rec), flush=True)
     if world > 1:
@@ -554,21 +690,25 @@ def run_gpu(args, spec) -> None:
         dist.destroy_process_group()
 
 
+def all_workloads():
+    return {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs(),
+            **synth.multi_query_configs(), **synth.paged_configs(), **synth.anchor_configs()}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    workloads = {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs(),
-                 **synth.multi_query_configs(), **synth.paged_configs()}
+    workloads = all_workloads()
     ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     spec = workloads[args.workload]
     if args.impl == "reference":
-        if isinstance(spec, synth.BifurcatedSpec):
-            raise SystemExit("the reference arm times the decode workloads")
+        if not isinstance(spec, synth.DecodeSpec) or spec.n_queries != 1 or spec.page_size:
+            raise SystemExit("the reference arm times the single-query decode workloads")
         run_reference(args, spec)
     else:
         run_gpu(args, spec)

@@ -12,6 +12,7 @@ import ctypes
 import os
 from typing import Optional, Sequence
 
+from . import _build
 from ._build import LIB, build  # noqa: F401
 
 TA_OK, TA_ERR_INVALID_ARG, TA_ERR_UNSUPPORTED, TA_ERR_WORKSPACE, TA_ERR_CUDA, TA_ERR_TIMEOUT = range(6)
@@ -21,6 +22,8 @@ TA_BF16, TA_F32 = 0, 1
 _DTYPES = {"bf16": TA_BF16, "f32": TA_F32}
 
 EXPORTED = [
+    "tree_attn_build_id",
+    "tree_attn_profile_events",
     "tree_attn_status_string",
     "tree_attn_last_cuda_error",
     "tree_attn_workspace_size",
@@ -33,6 +36,7 @@ EXPORTED = [
     "tree_attn_decode_bifurcated_ex",
     "tree_attn_check",
     "tree_attn_decode_noalloc",
+    "tree_attn_noalloc_check",
     "tree_attn_multi_workspace_size",
     "tree_attn_decode_multi_ex",
     "tree_attn_decode_multi",
@@ -40,6 +44,7 @@ EXPORTED = [
     "tree_attn_decode_paged",
     "tree_attn_merge_shards",
     "tree_attn_decode_multi_paged_ex",
+    "tree_attn_anchor_prefill",
 ]
 
 
@@ -78,12 +83,19 @@ _lib = None
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded library (raises if it has not been built)."""
+    """The loaded library.  Raises if it is missing, or if it was not built from the sources in
+    the tree (its build id, a hash of every source and header, differs from theirs)."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB):
             raise ImportError(f"{LIB} is missing: build it with exact_long_context_split_b200.build()")
         L = ctypes.CDLL(LIB)
+        L.tree_attn_build_id.argtypes = []
+        L.tree_attn_build_id.restype = ctypes.c_char_p
+        built, current = L.tree_attn_build_id().decode(), _build.source_hash()
+        if built != current:
+            raise ImportError(f"{LIB} was built from other sources (build id {built}, sources {current}): "
+                              "rebuild it with exact_long_context_split_b200.build()")
         vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
         pi64 = ctypes.POINTER(ctypes.c_int64)
         popt = ctypes.POINTER(ta_options)
@@ -91,6 +103,7 @@ def lib() -> ctypes.CDLL:
         sigs = {
             "tree_attn_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "tree_attn_last_cuda_error": ([], i32),
+            "tree_attn_profile_events": ([vp, vp], None),
             "tree_attn_workspace_size": ([pi64, i32, i32, i32, i32, ctypes.c_int, popt, psz], ctypes.c_int),
             "tree_attn_workspace_init": ([vp, sz, vp], ctypes.c_int),
             "tree_attn_decode": ([vp, vp, vp, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
@@ -110,6 +123,7 @@ def lib() -> ctypes.CDLL:
             ),
             "tree_attn_check": ([vp, vp], ctypes.c_int),
             "tree_attn_decode_noalloc": ([vp, vp, vp, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
+            "tree_attn_noalloc_check": ([vp], ctypes.c_int),
             "tree_attn_multi_workspace_size": ([pi64, i32, i32, i32, i32, i32, ctypes.c_int, popt, psz], ctypes.c_int),
             "tree_attn_decode_multi_ex": (
                 [ctypes.c_int, vp, vp, vp, pi64, i32, i32, i32, i32, i32, f32, vp, vp, popt, vp, sz, vp],
@@ -126,6 +140,8 @@ def lib() -> ctypes.CDLL:
                  vp],
                 ctypes.c_int,
             ),
+            "tree_attn_anchor_prefill": (
+                [vp, vp, vp, i64, i64, i32, i32, i32, f32, vp, vp, popt, vp, sz, vp], ctypes.c_int),
             "tree_attn_decode_paged": (
                 [vp, vp, vp, i64, i32, vp, i64, pi64, i32, i32, i32, i32, f32, vp, vp, vp], ctypes.c_int),
         }
@@ -179,6 +195,22 @@ def _check(status: int, where: str) -> None:
 # ----------------------------------------------------------------------------------------------
 # The C ABI, one Python function per entry point
 # ----------------------------------------------------------------------------------------------
+
+
+def tree_attn_build_id() -> str:
+    """Hash of the sources and headers the loaded library was built from."""
+    return lib().tree_attn_build_id().decode()
+
+
+def tree_attn_profile_events(start=None, stop=None) -> None:
+    """Record these CUDA events (torch.cuda.Event, recorded once so that they exist, or raw
+    cudaEvent_t handles) around the main kernel of every following call on this thread; no
+    arguments turns it off."""
+    def handle(e):
+        if e is None:
+            return None
+        return e if isinstance(e, int) else e.cuda_event
+    lib().tree_attn_profile_events(handle(start), handle(stop))
 
 
 def tree_attn_status_string(status: int) -> str:
@@ -271,6 +303,12 @@ def tree_attn_decode_noalloc(q, k_cache, v_cache, seqlens, n_q_heads, n_kv_heads
            "tree_attn_decode_noalloc")
 
 
+def tree_attn_noalloc_check(stream=None) -> int:
+    """Synchronise the stream and return the no-allocation scratch array's status (TA_OK or
+    TA_ERR_TIMEOUT); does not raise."""
+    return lib().tree_attn_noalloc_check(_stream(stream))
+
+
 def tree_attn_multi_workspace_size(seqlens, n_queries, n_q_heads, n_kv_heads, head_dim, dtype="bf16",
                                    opts=None) -> int:
     arr, n = _lens(seqlens)
@@ -343,3 +381,13 @@ def tree_attn_decode_multi_paged_ex(dtype, q, k_pages, v_pages, num_pages, page_
                                                  n_q_heads, n_kv_heads, head_dim, scale, _ptr(out), _ptr(lse),
                                                  _opts(opts), _ptr(workspace), workspace_bytes,
                                                  _stream(stream, q, out)), "tree_attn_decode_multi_paged_ex")
+
+
+def tree_attn_anchor_prefill(q, k, v, seq_len, block_size, n_q_heads, n_kv_heads, head_dim, scale, out, lse,
+                             opts, workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """Context encoding with anchor blocks: q, out [S][Hq][D], k, v [Hkv][S][D], lse [S][Hq]."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().tree_attn_anchor_prefill(_ptr(q), _ptr(k), _ptr(v), seq_len, block_size, n_q_heads, n_kv_heads,
+                                          head_dim, scale, _ptr(out), _ptr(lse), _opts(opts), _ptr(workspace),
+                                          workspace_bytes, _stream(stream, q, out)), "tree_attn_anchor_prefill")

@@ -44,7 +44,6 @@ constexpr int kBifVStages = 2;      // V ring depth (V frees a stage after O += 
 constexpr int kBifTmemCols = 512;   // S: 2 tiles x 128 columns; O: 2 tiles x 128 columns
 constexpr float kBifRescale = 8.0f;  // lazy rescaling threshold (log2 units)
 constexpr bool kBifPingPong = true;  // the two softmax warpgroups take turns on the exponentials
-constexpr int kBifPolyEvery = 0;     // every k-th pair of exponentials on the FMA pipe (0: none)
 
 
 struct BifSmem {
@@ -187,26 +186,6 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
   return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// 2^y for a pair, on the FMA pipe: y = j + f with j = rint(y) (the 1.5 * 2^23 rounding
-// trick) and f in [-1/2, 1/2]; 2^f from a degree-4 polynomial fitted here to the relative
-// error of 2^f on that interval (weighted least squares, max relative error 2.7e-6 with
-// float32 Horner evaluation); j is added to the exponent field.  y below -126 is clamped
-// (its power of two is below every value a softmax weight can contribute here).
-__device__ __forceinline__ float2 exp2_poly2(float2 y) {
-  y.x = fmaxf(y.x, -126.f);
-  y.y = fmaxf(y.y, -126.f);
-  const float2 t = __fadd2_rn(y, make_float2(12582912.f, 12582912.f));
-  const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), y);
-  float2 q = __ffma2_rn(make_float2(0.009570068679749966f, 0.009570068679749966f), f,
-                        make_float2(0.055917806923389435f, 0.055917806923389435f));
-  q = __ffma2_rn(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  q = __ffma2_rn(q, f, make_float2(0.6931218504905701f, 0.6931218504905701f));
-  q = __ffma2_rn(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // 3-input max / min (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -307,12 +286,7 @@ __device__ __forceinline__ void bif_exp_chunk(const float (&x)[32], uint32_t col
 #pragma unroll
   for (int c2 = 0; c2 < 16; ++c2) {
     const float2 y = __ffma2_rn(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, nm);
-    float2 pp;
-    constexpr int kMod = kBifPolyEvery > 0 ? kBifPolyEvery : 1;
-    if (kBifPolyEvery > 0 && c2 % kMod == kMod - 1)
-      pp = exp2_poly2(y);
-    else
-      pp = make_float2(ex2(y.x), ex2(y.y));
+    const float2 pp = make_float2(ex2(y.x), ex2(y.y));
     acc[c2 & 3] = __fadd2_rn(acc[c2 & 3], pp);
     const __half2 hv = __floats2half2_rn(pp.x, pp.y);
     h[c2] = *reinterpret_cast<const uint32_t*>(&hv);
@@ -395,21 +369,42 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const int lane = tid & 31;
   // The CTA's unit: its rows, its keys (a range of tensor-map rows) and its chunk of them.
   const bool multi = p.mode == 1;
-  const int chunk = multi ? blockIdx.x : blockIdx.y;
-  const int h = multi ? blockIdx.y : blockIdx.z;
+  const bool anchor = p.mode == 2;
+  const int chunk = multi ? blockIdx.x : (anchor ? 0 : blockIdx.y);
+  const int h = multi || anchor ? blockIdx.y : blockIdx.z;
   const int b = multi ? blockIdx.z : 0;
-  const int row0 = multi ? 0 : blockIdx.x * kBifMT * kBifRows;  // first row of this CTA in the unit
-  // Mode 0: M tile w holds rows row0 + 128 w + lane and reads every key tile.  Mode 1: both
-  // slots hold the unit's rows; slot w reads key tiles w, w + 2, ... ("split" slots).
-  const int n_mt = multi ? 1 : min(kBifMT, (p.rows_per_head - row0 + kBifRows - 1) / kBifRows);
-  const bool split = multi;
+  const int row0 = multi || anchor ? 0 : blockIdx.x * kBifMT * kBifRows;  // first row of this CTA in the unit
+  // Mode 0: M tile w holds rows row0 + 128 w + lane and reads every key tile.  Modes 1 and 2:
+  // both slots hold the unit's rows; slot w reads key tiles w, w + 2, ... ("split" slots).
+  const int n_mt = multi || anchor ? 1 : min(kBifMT, (p.rows_per_head - row0 + kBifRows - 1) / kBifRows);
+  const bool split = multi || anchor;
   const int n_slots = split ? kBifMT : n_mt;
-  const int64_t kv_len = multi ? p.kv_len[b] : p.prefix_len;
-  const int64_t kv_row0 = multi ? p.kv_row0[b] + h * kv_len : static_cast<int64_t>(h) * p.prefix_len;
-  const int q_tok0 = multi ? b * p.n_queries : 0;  // q row of the unit's first token / sample
+  // Mode 2: query tile qt (launched last tile first: the later blocks see the most keys) holds
+  // positions p0 .. p0 + n_pos - 1 of context block blk; its keys are the virtual sequence
+  // [anchor block ; own block up to its last position] (no anchor for the first block).
+  const int64_t qt = anchor ? static_cast<int64_t>(gridDim.x) - 1 - blockIdx.x : 0;
+  const int64_t p0 = qt * p.n_pos;
+  const int n_tok = anchor ? static_cast<int>(min(static_cast<int64_t>(p.n_pos), p.ctx_len - p0))
+                           : (multi ? p.n_queries : 1);  // query tokens of the unit
+  const int64_t blk = anchor ? p0 / p.block_size : 0;
+  const int64_t anchor_len = blk > 0 ? p.block_size : 0;  // keys of the anchor segment
+  const int64_t own0 = blk * p.block_size;                 // first key of the own segment
+  const int64_t kv_len = multi ? p.kv_len[b] : (anchor ? anchor_len + (p0 + n_tok - own0) : p.prefix_len);
+  const int64_t kv_row0 = multi ? p.kv_row0[b] + h * kv_len
+                                : static_cast<int64_t>(h) * (anchor ? p.ctx_len : p.prefix_len);
+  const int64_t q_tok0 = multi ? static_cast<int64_t>(b) * p.n_queries : p0;  // q row of the unit's first token
   const int64_t n_tiles = (kv_len + kBifKeys - 1) / kBifKeys;
   const int64_t j0 = chunk * n_tiles / p.n_chunks;
   const int n_t = static_cast<int>((chunk + 1) * n_tiles / p.n_chunks - j0);
+  // Tensor-map row of key tile t of the CTA's chunk (mode 2: the anchor segment, then the own
+  // one; block_size is a multiple of the tile, so no tile spans both).
+  auto tile_row = [&](int t) -> int {
+    const int64_t v = (j0 + t) * kBifKeys;
+    if (!anchor || v < anchor_len) return static_cast<int>(kv_row0 + v);
+    return static_cast<int>(kv_row0 + own0 + (v - anchor_len));
+  };
+  // Test hook: CTA (0, 0, 0) never loads this K tile, so the products that need it wait in vain.
+  const int skip_tile = (blockIdx.x | blockIdx.y | blockIdx.z) == 0 ? p.debug_skip_tile1 - 1 : -1;
 
   if (tid == 0) {
 #pragma unroll
@@ -454,11 +449,14 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     // whole warp, lane k issuing the k-th page segment's boxes.
     if (PAGED || lane == 0) {
       uint64_t pol;
-      asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-      int tk = 0, tv = 0;
+      if (anchor)  // every key tile is read by many query tiles: keep it in L2
+        asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+      else
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+      int fk[kBifKStages] = {}, fv[kBifVStages] = {};  // copies issued per stage
       if constexpr (!PAGED) {
         auto issue = [&](const CUtensorMap* map, uint8_t* dst, uint64_t* full, int t) {
-          const int y = static_cast<int>(kv_row0 + (j0 + t) * kBifKeys);
+          const int y = tile_row(t);
           mbar_arrive_expect_tx(full, 2 * kBifKeys * 128);
           tma_load_2d(dst, map, 0, y, full, pol);
           tma_load_2d(dst + kBifKeys * 128, map, 64, y, full, pol);
@@ -467,12 +465,14 @@ __global__ void __launch_bounds__(kBifThreads, 1)
         for (int t = 0; t < n_t && !*abort; ++t) {
           if (t >= kBifKStages && !bif_wait(&sm.k_empty[t % kBifKStages], ((t / kBifKStages) - 1) & 1, p, abort))
             break;
-          issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages], t);
-          ++tk;
+          if (t != skip_tile) {
+            issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages], t);
+            ++fk[t % kBifKStages];
+          }
           if (t >= kBifVStages && !bif_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1, p, abort))
             break;
           issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages], t);
-          ++tv;
+          ++fv[t % kBifVStages];
         }
       } else {
         // A tile is n_sub boxes of bs rows: one box of 128 rows of a contiguous cache, or one per
@@ -532,22 +532,21 @@ __global__ void __launch_bounds__(kBifThreads, 1)
           }
           if (t + 1 < n_t) fetch(t + 1);
           issue(&kmap, sm.k[t % kBifKStages][0], &sm.k_full[t % kBifKStages]);
-          ++tk;
+          ++fk[t % kBifKStages];
           if (t >= kBifVStages && !stage_wait(&sm.v_empty[t % kBifVStages], ((t / kBifVStages) - 1) & 1)) break;
           issue(&vmap, sm.v[t % kBifVStages][0], &sm.v_full[t % kBifVStages]);
-          ++tv;
+          ++fv[t % kBifVStages];
         }
       }
-      // Every issued copy lands before the CTA moves on (stage s holds tiles s, s + S, ...).
+      // Every issued copy lands before the CTA moves on: stage s completed one phase per copy
+      // issued to it, so the last of them has parity (count - 1) & 1.
       if (lane == 0) {
-        for (int s = 0; s < kBifKStages && s < tk; ++s) {
-          const int last = (tk - 1 - s) / kBifKStages;
-          if (!wait_phase(&sm.k_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
-        }
-        for (int s = 0; s < kBifVStages && s < tv; ++s) {
-          const int last = (tv - 1 - s) / kBifVStages;
-          if (!wait_phase(&sm.v_full[s], last & 1, p.wait_limit_ns, nullptr)) atomicCAS(p.err, 0, kErrBifWait);
-        }
+        for (int s = 0; s < kBifKStages; ++s)
+          if (fk[s] > 0 && !wait_phase(&sm.k_full[s], (fk[s] - 1) & 1, p.wait_limit_ns, nullptr))
+            atomicCAS(p.err, 0, kErrBifWait);
+        for (int s = 0; s < kBifVStages; ++s)
+          if (fv[s] > 0 && !wait_phase(&sm.v_full[s], (fv[s] - 1) & 1, p.wait_limit_ns, nullptr))
+            atomicCAS(p.err, 0, kErrBifWait);
       }
     }
     __syncwarp();
@@ -651,10 +650,10 @@ __global__ void __launch_bounds__(kBifThreads, 1)
     const uint32_t o_col = tmem + lane_base + 256 + w * 128;
     const int G = p.n_q_heads / p.n_kv_heads;
     const int row = split ? r : row0 + w * kBifRows + r;  // row of the unit's query matrix
-    const bool valid_row = row < p.rows_per_head;
-    // Keys at the end of the unit this row may not see (mode 1: query token j of n is
+    const bool valid_row = row < (anchor ? n_tok * G : p.rows_per_head);
+    // Keys at the end of the unit this row may not see (modes 1 and 2: query token j of n is
     // n - 1 - j positions before the last one).
-    const int lag = (multi && valid_row) ? p.n_queries - 1 - row / G : 0;
+    const int lag = (split && valid_row) ? n_tok - 1 - row / G : 0;
     if (!split || w == 0) {
       const int n = row / G, g = row % G;
       const uint4* src = reinterpret_cast<const uint4*>(
@@ -719,8 +718,54 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.p_full[w]);
     }
-    // The chunk's statistics of this row.
-    if (w < n_slots) {
+    if (anchor) {
+      // Mode 2: both slots hold the same rows over alternate key tiles.  Slot 1 publishes its
+      // (m, l) in shared memory (the second Q buffer, unused with split slots); slot 0 merges
+      // them with its own, reads both O accumulators from TMEM and writes the final row.
+      const int n1 = n_t / 2;  // key tiles of slot 1 (slot 0 has (n_t + 1) / 2 >= 1)
+      if (n_w > 0 && ok) {
+        ok = bif_wait(&sm.o_done[w], 0, p, abort);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      float* st = reinterpret_cast<float*>(sm.q[1][0]);
+      if (w == 1) {
+        st[r] = n1 > 0 ? m : -INFINITY;
+        st[kBifRows + r] = n1 > 0 ? l : 0.f;
+        st[2 * kBifRows + r] = ok ? 0.f : 1.f;
+        tc_fence_before();
+      }
+      named_barrier(1, 2 * kBifRows);
+      if (w == 0) {
+        tc_fence_after();
+        const float m1 = st[r], l1 = st[kBifRows + r];
+        const bool bad = !ok || st[2 * kBifRows + r] != 0.f;
+        const float M = fmaxf(m, m1);
+        const float a0 = (m == -INFINITY) ? 0.f : ex2(m - M);
+        const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+        const float L = l * a0 + l1 * a1;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float c0 = a0 * inv, c1 = a1 * inv;
+        const float nan = __int_as_float(0x7fc00000);
+        const int64_t orow = (q_tok0 + row / G) * p.n_q_heads + h * G + row % G;
+        float* dst = p.out + orow * kBifD;
+#pragma unroll 1
+        for (int q4 = 0; q4 < kBifD / 32; ++q4) {
+          float o[32], o1[32];
+          tmem_ld32(o_col + q4 * 32, o);  // slot 0 always has a tile (every query sees itself)
+          if (n1 > 0) tmem_ld32(o_col + 128 + q4 * 32, o1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = bad ? nan : (n1 > 0 ? o[c] * c0 + o1[c] * c1 : o[c] * c0);
+          if (valid_row) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dst + q4 * 32 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          }
+        }
+        if (valid_row) p.lse[orow] = bad ? nan : (L > 0.f ? (M + log2f(L)) * 0.693147180559945309f : -INFINITY);
+      }
+    } else if (w < n_slots) {
+      // The chunk's statistics of this row.
       // Mode 0: [chunk][KV head][row]; mode 1: [sequence, KV head][chunk][slot][row].
       const int64_t prow =
           multi ? ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.n_chunks + chunk) * kBifMT + w

@@ -48,7 +48,23 @@ struct BifParams {
   int64_t bt_stride;
   int64_t num_pages;
   int log2_page;
+  // mode 2: context encoding with anchor blocks (one context of ctx_len tokens); grid (query
+  //   tiles, KV heads); query tile qt holds positions qt * n_pos .. (n_pos = 128 / G, G heads
+  //   each, row j * G + g); the position at offset o of block i sees the anchor block (keys
+  //   [0, block_size), when i > 0) and keys [i * block_size, i * block_size + o]; the tensor maps
+  //   cover k, v [Hkv][ctx_len][D].  The CTA merges its two slots and writes out / lse itself.
+  int64_t ctx_len;
+  int64_t block_size;  // a multiple of kBifKeys
+  int n_pos;
+  float* out;          // [ctx_len][Hq][D]
+  float* lse;          // [ctx_len][Hq]
+  // Test hook: 0 off; t + 1: CTA (0, 0, 0) never loads K tile t of its chunk (the products that
+  // need it wait until the bounded wait runs out).
+  int debug_skip_tile1;
 };
+
+// The parameters and the two tensor maps share the 4 KB kernel-parameter space.
+static_assert(sizeof(BifParams) + 2 * sizeof(CUtensorMap) <= 4096, "kernel parameters must fit in 4 KB");
 
 // Dynamic shared memory of bif_prefix_kernel (the tile ring plus 1 KB for 1024-byte alignment).
 size_t bif_prefix_smem_bytes();

@@ -84,25 +84,8 @@ static_assert(sizeof(SplitParams) <= 4096, "kernel parameters must fit the 4 KB 
 // long sequences stream at the HBM roofline.  ShortTiles: 8 warps, 8 elements per lane,
 // 16 KB tiles (64 tokens at D = 128), a 4-deep ring: short sequences waste less of their
 // last tile.
-#ifndef TA_SPLIT_WARPS
-#define TA_SPLIT_WARPS 12
-#endif
-#ifndef TA_SPLIT_STAGES
-#define TA_SPLIT_STAGES 2
-#endif
-#ifndef TA_SPLIT_ELEMS
-#define TA_SPLIT_ELEMS 8
-#endif
-#ifndef TA_SPLIT_TILE_BYTES
-#define TA_SPLIT_TILE_BYTES 49152
-#endif
-#ifndef TA_SPLIT_KV_BARRIERS
-#define TA_SPLIT_KV_BARRIERS 0  // 1: separate "K landed" and "V landed" barriers per stage
-#endif
-
 struct LongTiles {
-  static constexpr int warps = TA_SPLIT_WARPS, stages = TA_SPLIT_STAGES, elems = TA_SPLIT_ELEMS,
-                       tile_bytes = TA_SPLIT_TILE_BYTES;
+  static constexpr int warps = 12, stages = 2, elems = 8, tile_bytes = 49152;
 };
 struct ShortTiles {
   static constexpr int warps = 8, stages = 4, elems = 8, tile_bytes = 16384;
@@ -161,8 +144,7 @@ struct SplitSmem {
   float mw[C::MERGE_BATCH][C::G];  // merge weights 2^(m_c - M)
   float mM[C::G];
   float mL[C::G];
-  uint64_t full[C::NSTAGE];   // K (and V, unless split) of the stage landed
-  uint64_t full_v[C::NSTAGE]; // V of the stage landed (split barriers only)
+  uint64_t full[C::NSTAGE];   // K and V (and q with a unit's first tile) of the stage landed
   uint64_t empty[C::NSTAGE];
   int is_last;
   int abort;
@@ -403,7 +385,6 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
 #pragma unroll
     for (int s = 0; s < C::NSTAGE; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.full_v[s], 1);
       mbar_init(&sm.empty[s], C::NCW);
     }
     sm.abort = 0;
@@ -441,8 +422,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
             const uint32_t bytes = static_cast<uint32_t>(nv) * C::ROW;
             constexpr uint32_t q_bytes = G * D * C::ELEM;
             const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
-            uint64_t* vbar = TA_SPLIT_KV_BARRIERS ? &sm.full_v[s] : &sm.full[s];
-            mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
+            mbar_arrive_expect_tx(&sm.full[s], 2 * bytes + (with_q ? q_bytes : 0));
             if (with_q) {
               // One copy per query token of the launch: its `heads` query heads are contiguous.
               const int heads = 1 << p.log2_heads;
@@ -455,11 +435,10 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
                 bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
               }
             }
-            if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(vbar, bytes);
             if (bytes != 0) {
               const int64_t off = p.kv_off[w.b] + (static_cast<int64_t>(w.h) * len + t0) * D;
               bulk_load(sm.k[s], reinterpret_cast<const T*>(p.k) + off, bytes, &sm.full[s], pol);
-              bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, vbar, pol);
+              bulk_load(sm.v[s], reinterpret_cast<const T*>(p.v) + off, bytes, &sm.full[s], pol);
             }
             ++fills[s];
           }
@@ -467,13 +446,12 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
         }
       }
     } else {
-      uint64_t* const vbar0 = TA_SPLIT_KV_BARRIERS ? sm.full_v : sm.full;
       // Stage s's expected bytes and the unit's q, which lands with the unit's first tile (one
       // copy per query token of the launch: its `heads` query heads are contiguous).  Lane 0.
       auto tile_header = [&](int s, int i, uint32_t bytes) {
         constexpr uint32_t q_bytes = G * D * C::ELEM;
         const bool with_q = (i == 0 || w.j == 0);  // the consumers switch to this unit here
-        mbar_arrive_expect_tx(&sm.full[s], (TA_SPLIT_KV_BARRIERS ? bytes : 2 * bytes) + (with_q ? q_bytes : 0));
+        mbar_arrive_expect_tx(&sm.full[s], 2 * bytes + (with_q ? q_bytes : 0));
         if (with_q) {
           const int heads = 1 << p.log2_heads;
           const uint32_t qb = static_cast<uint32_t>(heads) * D * C::ELEM;
@@ -484,7 +462,6 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
             bulk_load(sm.q[s] + jl * qb, qsrc, qb, &sm.full[s], pol);
           }
         }
-        if (TA_SPLIT_KV_BARRIERS) mbar_arrive_expect_tx(&vbar0[s], bytes);
       };
       auto stage_wait = [&](int s, int i) {  // lane 0: the stage's previous tile was consumed
         if (i >= C::NSTAGE && !wait_phase(&sm.empty[s], ((i / C::NSTAGE) - 1) & 1, p.wait_limit_ns, abort_flag)) {
@@ -554,7 +531,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
           const uint32_t nb = static_cast<uint32_t>(hi - lo) * C::ROW;
           const int64_t row = ((page * p.n_kv_heads + w.h) << p.log2_page) + (lo - first);
           bulk_load(sm.k[s] + (lo - t0) * C::ROW, reinterpret_cast<const T*>(p.k) + row * D, nb, &sm.full[s], pol);
-          bulk_load(sm.v[s] + (lo - t0) * C::ROW, reinterpret_cast<const T*>(p.v) + row * D, nb, &vbar0[s], pol);
+          bulk_load(sm.v[s] + (lo - t0) * C::ROW, reinterpret_cast<const T*>(p.v) + row * D, nb, &sm.full[s], pol);
         }
         page = page_n;
         n_pg = n_pg_n;
@@ -567,9 +544,6 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
 #pragma unroll
       for (int st = 0; st < C::NSTAGE; ++st) {
         if (fills[st] > 0 && !wait_phase(&sm.full[st], (fills[st] - 1) & 1, p.wait_limit_ns, nullptr))
-          atomicCAS(p.err, 0, kErrDrainWait);
-        if (TA_SPLIT_KV_BARRIERS && fills[st] > 0 &&
-            !wait_phase(&sm.full_v[st], (fills[st] - 1) & 1, p.wait_limit_ns, nullptr))
           atomicCAS(p.err, 0, kErrDrainWait);
       }
     }
@@ -840,17 +814,6 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
         for (int st = 0; st < C::STEPS; ++st) {
           pe[st] = (x[st] == -INFINITY) ? 0.f : ex2(x[st] - m);
           l += pe[st];
-        }
-        if (TA_SPLIT_KV_BARRIERS) {
-          bool vok = wait_phase(&sm.full_v[s], (i / C::NSTAGE) & 1, p.wait_limit_ns, abort_flag);
-          vok = __all_sync(kFull, vok);
-          if (!vok) {
-            if (lane == 0) {
-              if (!*abort_flag) atomicCAS(p.err, 0, kErrConsumerWait);
-              *abort_flag = 1;
-            }
-            ok = false;
-          }
         }
         // Phase C: o += p v for the same tokens.
 #pragma unroll

@@ -18,6 +18,23 @@ namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
 
+// Profiling hook (tree_attn_profile_events): events recorded on the call's stream around the
+// launches of the call's main kernel.
+thread_local cudaEvent_t g_prof_start = nullptr, g_prof_stop = nullptr;
+
+struct ProfileSpan {
+  cudaStream_t st;
+  bool open = false;
+  explicit ProfileSpan(cudaStream_t s) : st(s) {}
+  void begin() {
+    if (g_prof_start && !open) cudaEventRecord(g_prof_start, st);
+    open = true;
+  }
+  void end() {
+    if (g_prof_stop) cudaEventRecord(g_prof_stop, st);
+  }
+};
+
 constexpr size_t kAlign = 256;
 constexpr size_t kHeaderBytes = 256;  // error word and spare
 constexpr int64_t kDefaultWaitUs = 2000000;
@@ -225,6 +242,7 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
   int log2_heads = 0;
   while ((1 << (log2_heads + 1)) <= Hq / Hkv) ++log2_heads;
   const double s2 = static_cast<double>(scale) * 1.4426950408889634073599246810019;
+  ProfileSpan prof(st);
   for (const Group& g : plan.groups) {
     SplitParams p;
     std::memset(&p, 0, sizeof(p));
@@ -262,10 +280,12 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
       p.n_tiles[i] = g.n_tiles[i];
     }
     p.tile_off[g.nb] = g.tile_off[g.nb];
+    prof.begin();
     ki.fn<<<g.P, ki.threads, ki.smem, st>>>(p);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  prof.end();
   return TA_OK;
 }
 
@@ -457,6 +477,7 @@ ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, 
   if (s != TA_OK) return s;
   float* part = reinterpret_cast<float*>(base + kHeaderBytes);
   int64_t row0 = 0;  // tensor-map row of the group's first sequence
+  ProfileSpan prof(st);
   for (int b0 = 0; b0 < a.batch; b0 += kBifMaxSeq) {
     const int nb = std::min(kBifMaxSeq, a.batch - b0);
     BifParams bp;
@@ -480,14 +501,17 @@ ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, 
     bp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
     bp.mode = 1;
     bp.n_queries = n_queries;
+    bp.debug_skip_tile1 = (opts && opts->debug_skip_tile >= 0 && b0 == 0) ? opts->debug_skip_tile + 1 : 0;
     if (pc) {
       bp.block_table = pc->table + static_cast<int64_t>(b0) * pc->stride;
       bp.bt_stride = pc->stride;
       bp.num_pages = pc->num_pages;
       bp.log2_page = pc->log2_page;
     }
+    prof.begin();
     cudaError_t e = launch_bif_prefix(dim3(bp.n_chunks, a.Hkv, nb), kmap, vmap, bp, st);
     if (e != cudaSuccess) return cuda_fail(e);
+    if (b0 + kBifMaxSeq >= a.batch) prof.end();
     e = launch_merge_chunks(part, bp.n_chunks, a.Hkv, P.rows, n_queries, a.out + qrow0 * a.D, a.lse + qrow0, nb,
                             a.Hq, err, st);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -724,11 +748,19 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
       bpp.prefix_len = a.P;
       bpp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
       bpp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+      bpp.debug_skip_tile1 = (opts && opts->debug_skip_tile >= 0) ? opts->debug_skip_tile + 1 : 0;
       const dim3 grid(bp.mtiles, bp.chunks, a.Hkv);
+      ProfileSpan prof(st);
+      prof.begin();
       cudaError_t e = launch_bif_prefix(grid, kmap, vmap, bpp, st);
       if (e != cudaSuccess) return cuda_fail(e);
+      prof.end();
+      const cudaEvent_t saved_start = g_prof_start, saved_stop = g_prof_stop;
+      g_prof_start = g_prof_stop = nullptr;  // the suffix pass is not the main kernel here
       s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
                       base + bp.suffix_off, err, st);
+      g_prof_start = saved_start;
+      g_prof_stop = saved_stop;
       if (s != TA_OK) return s;
       e = launch_merge_prefix_suffix(bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse,
                                      a.N, a.Hq, err, st);
@@ -773,6 +805,11 @@ const char* tree_attn_status_string(ta_status s) {
 }
 
 int32_t tree_attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+void tree_attn_profile_events(void* start, void* stop) {
+  g_prof_start = static_cast<cudaEvent_t>(start);
+  g_prof_stop = static_cast<cudaEvent_t>(stop);
+}
 
 ta_status tree_attn_workspace_size(const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                    int32_t head_dim, ta_dtype dtype, const ta_options* opts, size_t* bytes) {
@@ -1082,16 +1119,21 @@ constexpr int kMaxDevices = 64;
 // address: the address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device, looked up once per device.
-ta_status noalloc_scratch_address(void** out) {
+// Device address of g_noalloc_scratch on the current device.  Looked up again on every call
+// made outside stream capture (so an address from before a device reset is never reused);
+// inside a capture the address from the last uncaptured call on this device is used.
+ta_status noalloc_scratch_address(cudaStream_t st, void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(st, &cap);
+  if (e != cudaSuccess) return cuda_fail(e);
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone || addr[dev] == nullptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -1118,10 +1160,10 @@ ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const voi
   const size_t need = kHeaderBytes + plan.body_bytes;
   if (need > kNoAllocScratchBytes) return TA_ERR_SCRATCH_LIMIT;
   void* ws = nullptr;
-  s = noalloc_scratch_address(&ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = noalloc_scratch_address(st, &ws);
   if (s != TA_OK) return s;
   // The array keeps whatever the previous call left: clear the error word and the tickets.
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   cudaError_t e = cudaMemsetAsync(base, 0, kHeaderBytes, st);
   for (const Group& g : plan.groups) {
@@ -1148,6 +1190,61 @@ ta_status tree_attn_merge_shards(const float* outs, const float* lses, int32_t n
   return TA_OK;
 }
 
+ta_status tree_attn_anchor_prefill(const void* q, const void* k, const void* v, int64_t seq_len, int64_t block_size,
+                                   int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale, float* out,
+                                   float* lse, const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  ta_status s = check_opts(opts);
+  if (s != TA_OK) return s;
+  if (seq_len < 0 || block_size <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0 ||
+      !std::isfinite(scale))
+    return TA_ERR_INVALID_ARG;
+  const int G = n_q_heads / n_kv_heads;
+  if (head_dim != kBifD || (G != 1 && G != 2 && G != 4 && G != 8) || block_size % kBifKeys != 0 ||
+      static_cast<int64_t>(n_kv_heads) * seq_len >= (int64_t(1) << 31))
+    return TA_ERR_UNSUPPORTED;
+  if (seq_len == 0) return TA_OK;
+  if (!q || !k || !v || !out || !lse) return TA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return TA_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, kAlign) || workspace_bytes < kHeaderBytes) return TA_ERR_WORKSPACE;
+  int sms = 0;
+  s = bif_tc_setup(&sms);
+  if (s != TA_OK) return s;
+  CUtensorMap kmap, vmap;
+  const int64_t rows = static_cast<int64_t>(n_kv_heads) * seq_len;
+  s = encode_cache_map(&kmap, k, rows, kBifKeys);
+  if (s != TA_OK) return s;
+  s = encode_cache_map(&vmap, v, rows, kBifKeys);
+  if (s != TA_OK) return s;
+  BifParams bp;
+  std::memset(&bp, 0, sizeof(bp));
+  bp.q = q;
+  bp.err = static_cast<int*>(workspace);
+  bp.n_samples = 1;
+  bp.n_q_heads = n_q_heads;
+  bp.n_kv_heads = n_kv_heads;
+  bp.n_pos = kBifRows / G;
+  bp.rows_per_head = kBifRows;
+  bp.n_chunks = 1;
+  bp.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634073599246810019);
+  bp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+  bp.mode = 2;
+  bp.ctx_len = seq_len;
+  bp.block_size = block_size;
+  bp.out = out;
+  bp.lse = lse;
+  bp.debug_skip_tile1 = (opts && opts->debug_skip_tile >= 0) ? opts->debug_skip_tile + 1 : 0;
+  const int64_t n_tiles = (seq_len + bp.n_pos - 1) / bp.n_pos;
+  ProfileSpan prof(static_cast<cudaStream_t>(stream));
+  prof.begin();
+  const cudaError_t e = launch_bif_prefix(dim3(static_cast<unsigned>(n_tiles), n_kv_heads, 1), kmap, vmap, bp,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  prof.end();
+  return TA_OK;
+}
+
 ta_status tree_attn_check(const void* ws, void* stream) {
   if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
@@ -1157,6 +1254,16 @@ ta_status tree_attn_check(const void* ws, void* stream) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (word == 0) return TA_OK;
   return word == kErrBadPage ? TA_ERR_BAD_PAGE : TA_ERR_TIMEOUT;
+}
+
+ta_status tree_attn_noalloc_check(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  void* ws = nullptr;
+  const ta_status s = noalloc_scratch_address(st, &ws);
+  if (s != TA_OK) return s;
+  return tree_attn_check(ws, stream);
 }
 
 }  // extern "C"

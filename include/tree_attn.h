@@ -80,7 +80,8 @@ typedef struct {
   int32_t wait_limit_us;   /* 0: 2,000,000 us.  Bound on every wait inside a kernel; on expiry the
                               kernel records TA_ERR_TIMEOUT in the workspace and returns */
   int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
-                              consumers' wait runs out (no fault: the data simply never arrives) */
+                              consumers' wait runs out (no fault: the data simply never arrives).
+                              Tensor-core passes: CTA (0, 0, 0) never loads this K tile */
   int32_t prefix_path;     /* bifurcated and multi-query calls.  Bifurcated: 0 automatic (tensor-
                               core prefix pass when head_dim is 128 and the prefix is not empty);
                               1 tensor-core pass (TA_ERR_UNSUPPORTED if not possible); 2 split-KV
@@ -91,6 +92,26 @@ typedef struct {
                               sequence is under 1024 tokens); 1: long tiles; 2: short tiles */
   int32_t reserved[3];     /* must be 0 */
 } ta_options;
+
+/*
+ * Build identity (no counterpart in the pages): a hash of every library source file and
+ * public header, and of the compiler flags, that this binary was built from (static storage).
+ * Lets a caller or a test check that the loaded library matches the sources it reads.
+ */
+const char* tree_attn_build_id(void);
+
+/*
+ * Profiling hook (no counterpart in the pages).  While set (non-NULL, on this host thread),
+ * every call records `start` (a cudaEvent_t) on its stream immediately before the first launch
+ * of its main kernel and `stop` immediately after the last one, so the caller can time that
+ * kernel alone with cudaEventElapsedTime.  The main kernel is the split-KV kernel for decode
+ * (contiguous or paged; every pass of a multi-query call), the tensor-core kernel for the
+ * shared-prefix, multi-query tensor-core and context-encoding calls (the shared-prefix call's
+ * suffix pass and every merge launch fall outside the span, except the merges between the
+ * tensor-core launches of multi-query calls over more than 128 sequences).  NULL, NULL turns
+ * it off.  The library never creates, waits on or destroys the events.
+ */
+void tree_attn_profile_events(void* start, void* stop);
 
 /* A short English name of a status code (static storage). */
 const char* tree_attn_status_string(ta_status status);
@@ -216,19 +237,31 @@ ta_status tree_attn_decode_bifurcated_ex(const void* q, const void* k_prefix, co
  * a fixed 4 MiB scratch array that the library keeps in device memory (every GPU
  * that loads the library holds it until the process exits).
  *
- * The first call on each device looks up that array's device address (once per
- * device, with the device current); make that first call before any stream
- * capture.  Every call zero-fills the array's merge tickets and error word on
- * `stream` before its kernel runs.  All calls share the one array, so calls that
- * overlap on the GPU (two streams, two host threads) race and must be
- * serialised by the caller.  A problem whose workspace would exceed 4 MiB
- * (grid + B*Hkv partial slots of G*(D+2) floats, plus a ticket per sequence and
- * KV head) returns TA_ERR_SCRATCH_LIMIT before anything is launched.  Other
- * arguments and statuses as tree_attn_decode.
+ * Each call made outside stream capture looks up that array's device address on
+ * the current device (with that device current); a call inside a capture reuses the
+ * address of the last uncaptured call on the device, so make one call on each
+ * device before any stream capture.  Every call zero-fills the array's merge
+ * tickets and error word on `stream` before its kernel runs.  All calls share the
+ * one array, so calls that overlap on the GPU (two streams, two host threads) race
+ * and must be serialised by the caller.  A problem whose workspace would exceed
+ * 4 MiB (grid + B*Hkv partial slots of G*(D+2) floats, plus a ticket per sequence
+ * and KV head) returns TA_ERR_SCRATCH_LIMIT before anything is launched.  Other
+ * arguments and statuses as tree_attn_decode.  Device-side errors (a bounded wait
+ * that ran out: the affected outputs are NaN) are recorded in the array's error
+ * word, which tree_attn_noalloc_check reads.
  */
 ta_status tree_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int64_t* seqlens,
                                    int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
                                    float scale, float* out, float* lse, void* stream);
+
+/*
+ * Synchronise `stream` and read the error word of tree_attn_decode_noalloc's scratch array
+ * on the current device (no counterpart in the pages): TA_OK, TA_ERR_TIMEOUT if a bounded
+ * wait inside the last call's kernel ran out (its affected outputs are NaN), or TA_ERR_CUDA.
+ * Allocates nothing.  Like the calls themselves, it must not overlap another no-allocation
+ * call on the device.
+ */
+ta_status tree_attn_noalloc_check(void* stream);
 
 /*
  * Decode over a paged KV cache, after the attention-acceleration concept page
@@ -290,6 +323,29 @@ ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void*
  */
 ta_status tree_attn_merge_shards(const float* outs, const float* lses, int32_t n_shards, int64_t rows,
                                  int32_t head_dim, float* out, float* lse, void* stream);
+
+/*
+ * Context encoding with anchor blocks, after the Star Attention article (tiaojiaomugou.com,
+ * "Two-phase inference under Star Attention", "Phase 1: context encoding"): the context is cut
+ * into blocks of `block_size` tokens, every block after the first is prefixed with the first
+ * block (the anchor block), and each block attends causally over [anchor ; itself].  Exact
+ * softmax attention under that mask, for every position p of one context of `seq_len` tokens:
+ * with i = p / block_size, position p attends to keys [0, p] when i = 0 and to keys
+ * [0, block_size) and [i * block_size, p] when i > 0 (query head h reads KV head h / G).
+ *   q    [seq_len][Hq][D] bf16        k, v  [Hkv][seq_len][D] bf16
+ *   out  [seq_len][Hq][D] f32 (16-byte aligned)   lse [seq_len][Hq] f32
+ * Supported: head_dim 128, G = Hq / Hkv in {1, 2, 4, 8}, block_size a positive multiple of 128,
+ * Hkv * seq_len < 2^31; others -> TA_ERR_UNSUPPORTED.  A block_size >= seq_len is plain causal
+ * attention.  Runs on the tensor cores (tcgen05): one CTA per (query tile of 128 / G positions x
+ * G heads, KV head), S = Q K^T and O = P V with TMEM accumulators over the tile's anchor and own
+ * keys.  `workspace`: at least 256 bytes, 256-byte aligned, zero-filled before first use (its
+ * first word is the error word tree_attn_check reads: a bounded wait that ran out makes the
+ * affected rows NaN).  Other rules (options, statuses, asynchrony) as tree_attn_decode_ex.
+ */
+ta_status tree_attn_anchor_prefill(const void* q, const void* k, const void* v, int64_t seq_len, int64_t block_size,
+                                   int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, float scale, float* out,
+                                   float* lse, const ta_options* opts, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /*
  * Synchronise `stream` and read the workspace's error word: TA_OK, or

@@ -319,13 +319,11 @@ def bifurcated_attention(q, k_prefix, v_prefix, prefix_len: int, k_suffix, v_suf
     for n in sorted({p[0] for p in todo}):
         Ks = to_f64(sequence_block(k_suffix, suffix_lens, n, Hkv, D), dtype)
         Vs = to_f64(sequence_block(v_suffix, suffix_lens, n, Hkv, D), dtype)
-        for (nn, h) in todo:
-            if nn != n:
-                continue
-            g = h // G
+        for g in sorted({h // G for (nn, h) in todo if nn == n}):
+            heads = [h for (nn, h) in todo if nn == n and h // G == g]
             K = np.concatenate([Kp[g], Ks[g]], axis=0)
             V = np.concatenate([Vp[g], Vs[g]], axis=0)
-            out[n, h], lse[n, h] = attention_one(qf[n, h], K, V, scale)
+            out[n, heads], lse[n, heads] = attention_heads_cache(qf[n, heads], K, V, scale, "f64")
     return out, lse
 
 

@@ -301,3 +301,61 @@ def make_bifurcated_inputs(spec: BifurcatedSpec) -> Dict[str, np.ndarray]:
         "v_suffix": normal_bf16(spec.seed, TID_V_SUFFIX, n_suffix),
         "suffix_lens": np.asarray(spec.suffix_lens, dtype=np.int64),
     }
+
+
+@dataclasses.dataclass(frozen=True)
+class AnchorSpec:
+    """Context encoding with anchor blocks: one context of seq_len tokens in blocks of
+    block_size, every block after the first prefixed with the first (anchor) block."""
+
+    name: str
+    seq_len: int
+    block_size: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return float(np.float32(1.0 / math.sqrt(self.head_dim)))
+
+    @property
+    def visible_keys(self) -> int:
+        """Sum over positions of the keys each one attends to (anchor block plus its own block up
+        to itself; the first block has no anchor)."""
+        S, B = self.seq_len, self.block_size
+        total = 0
+        for i0 in range(0, S, B):
+            L = min(B, S - i0)
+            total += L * (B if i0 > 0 else 0) + L * (L + 1) // 2
+        return total
+
+    @property
+    def flops(self) -> int:
+        """Algorithmic FLOPs: for every (position, query head) and visible key, a D-long dot
+        product for the score and a D-long multiply-add for the output (2 D each)."""
+        return 4 * self.head_dim * self.n_q_heads * self.visible_keys
+
+    @property
+    def kv_bytes(self) -> int:
+        return 2 * 2 * self.n_kv_heads * self.seq_len * self.head_dim
+
+
+def anchor_configs() -> Dict[str, AnchorSpec]:
+    """Llama-3-8B-shaped context encoding (32/8 heads, head_dim 128) with the block a quarter of
+    the context: 32K tokens in 8K blocks, and 128K tokens in 32K blocks."""
+    return {
+        "star_prefill_32k": AnchorSpec("star_prefill_32k", 32_768, 8_192, 32, 8, 128, seed=9),
+        "star_prefill_128k": AnchorSpec("star_prefill_128k", 131_072, 32_768, 32, 8, 128, seed=10),
+    }
+
+
+def make_anchor_inputs(spec: AnchorSpec) -> Dict[str, np.ndarray]:
+    """q [S][Hq][D], k and v [Hkv][S][D], bf16 bits, ~N(0,1)."""
+    S, Hq, Hkv, D = spec.seq_len, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
+    return {
+        "q": normal_bf16(spec.seed, TID_Q, S * Hq * D).reshape(S, Hq, D),
+        "k": normal_bf16(spec.seed, TID_K, Hkv * S * D),
+        "v": normal_bf16(spec.seed, TID_V, Hkv * S * D),
+    }

@@ -93,20 +93,45 @@ def test_tensor_core_prefix_unsupported_shape():
 
 
 def test_bifurcated_equals_plain_decode_of_concatenation():
-    """Exactness of the split: the GPU bifurcated result matches the GPU plain decode over
-    [prefix ; suffix_n] (both checked against the oracle)."""
+    """Exactness of the split: the GPU bifurcated result (prefix and suffix parts merged) matches
+    the GPU plain decode of each sample's concatenated cache [prefix ; suffix_n] within the
+    tolerance, and both match the oracle."""
     sp = synth.BifurcatedSpec("case", 3000, [7, 300], 8, 2, 128, seed=22)
     inp = synth.make_bifurcated_inputs(sp)
     out, lse = bif_gpu(inp, sp)
     ref = oracle_bif(inp, sp)
     compare(out, lse, *ref)
+    # the same samples as plain decode: sequence n's cache is [prefix ; suffix_n] per KV head
+    P, Hkv, D, lens = sp.prefix_len, sp.n_kv_heads, sp.head_dim, list(sp.suffix_lens)
+    kp = inp["k_prefix"].reshape(Hkv, P, D)
+    vp = inp["v_prefix"].reshape(Hkv, P, D)
+    ks, vs, off = [], [], 0
+    for S in lens:
+        ks.append(np.concatenate([kp, inp["k_suffix"][off:off + Hkv * S * D].reshape(Hkv, S, D)], axis=1))
+        vs.append(np.concatenate([vp, inp["v_suffix"][off:off + Hkv * S * D].reshape(Hkv, S, D)], axis=1))
+        off += Hkv * S * D
+    dec = synth.DecodeSpec("concat", [P + S for S in lens], sp.n_q_heads, Hkv, D, seed=22)
+    dinp = {"q": inp["q"], "k": np.concatenate([x.reshape(-1) for x in ks]),
+            "v": np.concatenate([x.reshape(-1) for x in vs])}
+    from gpu_util import decode_gpu
+
+    plain_out, plain_lse = decode_gpu(dinp, dec)
+    compare(plain_out, plain_lse, *ref)
+    compare(out, lse, plain_out.astype(np.float64), plain_lse.astype(np.float64))
 
 
 @pytest.mark.parametrize("prefix_path", [1, 2])
 def test_bifurcated_config_sampled(prefix_path):
+    """The shared-prefix workload (64 samples, 65,536 + 256 tokens): every query head of 16
+    samples spread over the batch."""
+    from gpu_util import oracle_parallel
+
     sp = synth.bifurcated_configs()["shared_prefix"]
     inp = synth.make_bifurcated_inputs(sp)
     out, lse = bif_gpu(inp, sp, "ex", prefix_path)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
-    pairs = [(0, 0), (17, 9), (40, 22), (63, 31)]
-    compare(out, lse, *oracle_bif(inp, sp, pairs=pairs), pairs=pairs)
+    samples = list(range(0, sp.n_samples, 4)) + [sp.n_samples - 1]
+    tasks = [[(n, h) for h in range(sp.n_q_heads)] for n in samples]
+    ref_out, ref_lse = oracle_parallel(lambda pairs: oracle_bif(inp, sp, pairs=pairs), tasks, workers=4)
+    pairs = [p for t in tasks for p in t]
+    compare(out, lse, ref_out, ref_lse, pairs=pairs)

@@ -1,7 +1,6 @@
 """GPU parity of split decode attention against the CPU oracle, through the C ABI.
 
-Small and medium cases are compared on every output; the full-size workloads on sampled
-(sequence, head) rows that the oracle computes one by one.
+Every case, the full-size workloads included, is compared on every output row.
 """
 import numpy as np
 import pytest
@@ -159,22 +158,28 @@ def test_config_llama3_8b_gqa_full():
     compare(out, lse, *oracle_of(inp, sp))
 
 
-def _sampled(name, pairs):
+def _full_size(name, workers=0):
+    """A full-size workload: every (sequence, query head) row against the oracle, the row groups
+    of one (sequence, KV head) computed side by side on the host cores."""
+    from gpu_util import oracle_parallel
+
     sp = synth.decode_configs()[name]
     inp = synth.make_decode_inputs(sp)
     out, lse = decode_gpu(inp, sp)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
-    ref_out, ref_lse = oracle_of(inp, sp, pairs=pairs)
-    return compare(out, lse, ref_out, ref_lse, pairs=pairs)
+    G = sp.n_q_heads // sp.n_kv_heads
+    tasks = [[(b, g * G + i) for i in range(G)] for b in range(sp.batch) for g in range(sp.n_kv_heads)]
+    ref_out, ref_lse = oracle_parallel(lambda pairs: oracle_of(inp, sp, pairs=pairs), tasks, workers)
+    return compare(out, lse, ref_out, ref_lse)
 
 
-def test_config_long_1m_sampled():
-    _sampled("long_1m", [(0, 0), (0, 5), (0, 14), (0, 31)])
+def test_config_long_1m_all_rows():
+    _full_size("long_1m")
 
 
-def test_config_extreme_5m_sampled():
-    _sampled("extreme_5m", [(0, 3), (0, 28)])
+def test_config_extreme_5m_all_rows():
+    _full_size("extreme_5m", workers=4)
 
 
-def test_config_extreme_ragged_sampled():
-    _sampled("extreme_ragged", [(0, 0), (1, 9), (2, 17), (3, 31), (3, 0)])
+def test_config_extreme_ragged_all_rows():
+    _full_size("extreme_ragged", workers=4)

@@ -154,15 +154,12 @@ def test_allocating_entry_point():
 
 @pytest.mark.parametrize("name", ["spec_decode_2", "spec_decode_4"])
 def test_spec_decode_workload_sampled(name):
-    """The bench workloads (8 x 32K tokens, 32/8 heads) on sampled rows, every query token."""
+    """The bench workloads (8 x 32K tokens, 32/8 heads): every row of every query token."""
     sp = synth.multi_query_configs()[name]
     inp = synth.make_decode_inputs(sp)
     out, lse = multi_gpu(inp, sp)
-    r = np.random.default_rng(3)
-    rows = sorted({(int(r.integers(sp.batch)), j, int(r.integers(sp.n_q_heads))) for j in range(sp.n_queries)
-                   for _ in range(3)})
-    check(out, lse, inp, sp, rows=rows)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    check(out, lse, inp, sp)
 
 
 def test_invalid_arguments():

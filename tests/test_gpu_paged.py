@@ -137,8 +137,8 @@ def test_invalid_page_size():
         assert e.value.status == ta.TA_ERR_INVALID_ARG
 
 
-def test_long_1m_paged_sampled():
-    """The bench workload: 1M tokens in 16-token blocks at random places, sampled rows."""
+def test_long_1m_paged_all_rows():
+    """The bench workload: 1M tokens in 16-token blocks at random places, every row."""
     import torch
 
     import exact_long_context_split_b200 as ta
@@ -163,10 +163,16 @@ def test_long_1m_paged_sampled():
                                  sp.scale, out, lse, None, ws)
     assert ta.tree_attn_check(ws) == ta.TA_OK
     out, lse = out.cpu().numpy(), lse.cpu().numpy()
-    pairs = [(0, 0), (0, 13), (0, 31)]
-    ref_out, ref_lse = oracle.decode_attention(inp["q"], inp["k"], inp["v"], sp.seqlens, 32, Hkv, D, sp.scale,
-                                               pairs=pairs)
-    compare(out, lse, ref_out, ref_lse, pairs=pairs)
+    # the paged cache holds the contiguous cache's rows (pinned on the CPU), so the oracle reads
+    # the contiguous one: every row, a KV head's query heads per task
+    from gpu_util import oracle_parallel
+
+    G = 32 // Hkv
+    tasks = [[(0, g * G + i) for i in range(G)] for g in range(Hkv)]
+    ref_out, ref_lse = oracle_parallel(
+        lambda pairs: oracle.decode_attention(inp["q"], inp["k"], inp["v"], sp.seqlens, 32, Hkv, D, sp.scale,
+                                              pairs=pairs), tasks)
+    compare(out, lse, ref_out, ref_lse)
 
 
 # Several query tokens per sequence over a paged cache: the tensor-core form (one TMA box per

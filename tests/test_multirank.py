@@ -64,13 +64,54 @@ def test_record_fields():
     import synth
 
     spec = synth.decode_configs()["long_1m"]
-    rec = bench.make_record(value=1.0, n_gpus=2, steps=3, warmup=3, ms_per_step=0.5, spec=spec, dtype="bf16",
-                            extra={"gpu_launches": 3})
+    rec = bench.make_record(metric=bench.METRIC, unit=bench.UNIT, value=1.0, n_gpus=2, steps=3, warmup=3,
+                            ms_per_step=0.5, spec=spec, dtype="bf16", extra={"gpu_launches": 3})
     for key in ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
                 "vs_baseline", "dtype", "data", "config", "gpu_launches"]:
         assert key in rec
     assert rec["scaling"] == "weak" and rec["config"]["workload"] == "long_1m"
     json.dumps(rec)
+
+
+def test_record_config_of_every_workload():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for name, spec in bench.all_workloads().items():
+        cfg = bench.workload_config(spec, 1)
+        assert cfg["workload"] == name and cfg["kv_bytes_per_step"] == spec.kv_bytes
+        assert ("no flush" in cfg["l2"]) == (spec.kv_bytes > 2 * 126e6)
+
+
+def test_reference_arm_runs_full_steps_on_the_host():
+    """The reference arm times the oracle on every row of each step, threaded over rows."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300,
+                       env=dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0"))
+    assert r.returncode == 0, r.stderr
+    rec = json.loads(r.stdout.strip().splitlines()[-1])
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["gpu_launches"] == 0
+    assert "all 1 (sequence, query head) rows" in rec["cpu_baseline"]["sample"]
+    assert rec["cpu_baseline"]["cores"] == 1 and rec["cpu_baseline"]["host_cores"] >= 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_sampler_edges_without_nvml():
+    """Without NVML the sampler reports why, and the bench still gets a summary."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    c = bench.ClockSampler(0)
+    c.err = "nvml: not available"
+    c.start()
+    c.stop()
+    assert c.summary()["reasons"] == ["nvml: not available"] and c.summary()["samples"] == 0
+    c = bench.ClockSampler(0)
+    c.max_mhz = 1965
+    c.samples = [(1.0, 1965, 0), (2.0, 1800, 0x4), (3.5, 1965, 0)]
+    c.window = [1.0005, 3.4995]
+    s = c.summary()
+    assert s["samples"] == 3 and s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] == 1965
 
 
 def _sharded_rank(rank, world, port, q):
