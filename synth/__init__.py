@@ -205,10 +205,12 @@ def multi_query_configs() -> Dict[str, DecodeSpec]:
     }
 
 
-def capture_configs() -> Dict[str, DecodeSpec]:
-    """Smaller versions of the long-context workload for profiler captures (same recipe,
-    1/4 of the length: 1.07 GB of K/V, still far larger than the 126 MB L2)."""
-    return {"long_256k": DecodeSpec("long_256k", [262_144], 32, 8, 128, seed=3, spike_frac=0.001)}
+def capture_configs():
+    """Smaller versions of workloads for profiler captures: the long-context decode at 1/4 of the
+    length (same recipe, 1.07 GB of K/V, still far larger than the 126 MB L2), and context
+    encoding over 8K tokens in 2K blocks."""
+    return {"long_256k": DecodeSpec("long_256k", [262_144], 32, 8, 128, seed=3, spike_frac=0.001),
+            "star_prefill_8k": AnchorSpec("star_prefill_8k", 8_192, 2_048, 32, 8, 128, seed=11)}
 
 
 def bifurcated_configs() -> Dict[str, BifurcatedSpec]:
