@@ -32,14 +32,4 @@ cudaError_t launch_merge_chunks(const float* part, int n_chunks, int n_kv_heads,
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,
-                                       const float* out_s, const float* lse_s, float* out, float* lse,
-                                       int n_samples, int n_q_heads, const int* err, cudaStream_t st) {
-  const int64_t n = static_cast<int64_t>(n_samples) * n_q_heads * (kBifD / 4);  // one thread per 4 columns
-  if (n == 0) return cudaSuccess;
-  merge_prefix_suffix_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
-      part, n_chunks, n_kv_heads, rows_per_head, out_s, lse_s, out, lse, n_samples, n_q_heads, err);
-  return cudaGetLastError();
-}
-
 }  // namespace ta

@@ -11,7 +11,7 @@
 // tiles of keys, running max m and sum l, output rescaled when m grows).
 //
 // Each CTA writes per row the statistics (m in log2 units, l, unnormalised o) of its
-// chunk; merge_prefix_suffix_kernel combines the chunks with the suffix part.
+// chunk; the suffix pass (split kernel) folds them into each row as it writes the result.
 //
 // One CTA owns up to 256 rows (two M tiles of 128) and a contiguous chunk of 128-key
 // tiles of the context; both M tiles consume every K/V tile it loads.
@@ -667,6 +667,10 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       fence_proxy_async_smem();
     }
     mbar_arrive(&sm.q_ready);
+    // A warp none of whose rows is real (few rows per unit, a partial last tile) skips the
+    // scores' max and exponentials and the rescaling: its Q rows are zero, so its S rows, and
+    // the P rows read over them, are zero.  It still takes every wait and arrival in order.
+    const bool active = __any_sync(0xffffffffu, valid_row);
     const float sc = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = w < n_slots;
@@ -683,7 +687,7 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       // tcgen05.ld is warp-collective: a warp takes the masked path if any of its rows needs it.
       const bool full = __all_sync(0xffffffffu, nvalid >= kBifKeys);
       // Pass 1: the tile's scaled row max, streamed from TMEM.
-      const float tmax = full ? bif_tile_max(s_col, sc) : bif_tile_max_partial(s_col, sc, nvalid);
+      const float tmax = !active ? -INFINITY : (full ? bif_tile_max(s_col, sc) : bif_tile_max_partial(s_col, sc, nvalid));
       const bool need = tmax > m + kBifRescale;
       const float mn = need ? tmax : m;
       // Ping-pong: M tile 1's exponentials of key tile i follow M tile 0's, and M tile 0's of
@@ -697,11 +701,11 @@ __global__ void __launch_bounds__(kBifThreads, 1)
       }
       // Pass 2: p = 2^(x s - m), summed in fp32, written back as fp16 pairs over the first 64
       // columns of S (P overwrites only columns whose scores were already read).
-      const float rs = full ? bif_tile_exp(s_col, sc, mn) : bif_tile_exp_partial(s_col, sc, mn, nvalid);
+      const float rs = !active ? 0.f : (full ? bif_tile_exp(s_col, sc, mn) : bif_tile_exp_partial(s_col, sc, mn, nvalid));
       if (pingpong) mbar_arrive(&sm.turn[1 - w]);
       const float alpha = (need && m != -INFINITY) ? ex2(m - mn) : 1.f;
       // O holds tiles 0..i-1 and P(i - 1) V(i - 1) is complete: rescale it when m grew.
-      if (__any_sync(0xffffffffu, need && i >= 1)) {
+      if (active && __any_sync(0xffffffffu, need && i >= 1)) {
 #pragma unroll
         for (int q4 = 0; q4 < kBifD / 32; ++q4) {
           float o[32];
@@ -855,59 +859,6 @@ __global__ void __launch_bounds__(128) merge_chunks_kernel(const float* __restri
     lv = (M + log2f(L)) * 0.693147180559945309f;
   }
   if (*reinterpret_cast<const volatile int*>(err) != 0) {
-    const float nan = __int_as_float(0x7fc00000);
-    ov = make_float4(nan, nan, nan, nan);
-    lv = nan;
-  }
-  *reinterpret_cast<float4*>(out + rq * kBifD + d4) = ov;
-  if (d4 == 0) lse[rq] = lv;
-}
-
-// Suffix part given normalised (out_s, lse_s); it enters as m = lse_s log2(e), l = 1, o = out_s.
-// One thread per 4 columns of an output row.  One online pass over the chunks (the running
-// max moves only when a chunk's m exceeds it): each chunk's loads depend on nothing computed
-// before them, so an unrolled group of chunks has all its loads in flight at once.
-__global__ void __launch_bounds__(128) merge_prefix_suffix_kernel(
-    const float* __restrict__ part, int n_chunks, int n_kv_heads, int rows_per_head, const float* __restrict__ out_s,
-    const float* __restrict__ lse_s, float* __restrict__ out, float* __restrict__ lse, int n_samples, int n_q_heads,
-    const int* __restrict__ err) {
-  constexpr int Q = kBifD / 4;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(n_samples) * n_q_heads * Q;
-  if (i >= total) return;
-  const int d4 = static_cast<int>(i % Q) * 4;
-  const int64_t rq = i / Q;  // n * Hq + hq
-  const int n = static_cast<int>(rq / n_q_heads), hq = static_cast<int>(rq % n_q_heads);
-  const int G = n_q_heads / n_kv_heads;
-  const int h = hq / G, g = hq % G;
-  const float* base = part + (static_cast<int64_t>(h) * rows_per_head + n * G + g) * kBifPartRow;
-  const int64_t stride = static_cast<int64_t>(n_kv_heads) * rows_per_head * kBifPartRow;
-  const float ls = lse_s[rq];
-  float M = (ls == -INFINITY) ? -INFINITY : ls * 1.44269504088896340736f;
-  float L = (ls == -INFINITY) ? 0.f : 1.f;
-  float4 O = (ls == -INFINITY) ? make_float4(0.f, 0.f, 0.f, 0.f)
-                               : *reinterpret_cast<const float4*>(out_s + rq * kBifD + d4);
-#pragma unroll 9
-  for (int c = 0; c < n_chunks; ++c) {
-    const float* pc = base + c * stride;
-    const float2 ml = *reinterpret_cast<const float2*>(pc);
-    const float4 o = *reinterpret_cast<const float4*>(pc + 4 + d4);
-    // No branch: an empty chunk (m = -inf) gets weight 0, so the loads of the whole unrolled
-    // group issue together.
-    const float Mn = fmaxf(M, ml.x);
-    const float a = (M == -INFINITY) ? 0.f : ex2(M - Mn);
-    const float b = (ml.x == -INFINITY) ? 0.f : ex2(ml.x - Mn);
-    L = L * a + ml.y * b;
-    O = make_float4(O.x * a + o.x * b, O.y * a + o.y * b, O.z * a + o.z * b, O.w * a + o.w * b);
-    M = Mn;
-  }
-  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lv = -INFINITY;
-  if (L > 0.f) {
-    ov = make_float4(O.x / L, O.y / L, O.z / L, O.w / L);
-    lv = (M + log2f(L)) * 0.693147180559945309f;
-  }
-  if (*reinterpret_cast<const volatile int*>(err) != 0 || ls != ls) {
     const float nan = __int_as_float(0x7fc00000);
     ov = make_float4(nan, nan, nan, nan);
     lv = nan;

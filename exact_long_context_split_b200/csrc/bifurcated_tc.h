@@ -80,9 +80,4 @@ cudaError_t launch_bif_prefix(dim3 grid, const CUtensorMap& kmap, const CUtensor
 cudaError_t launch_merge_chunks(const float* part, int n_chunks, int n_kv_heads, int rows_per_head, int n_queries,
                                 float* out, float* lse, int batch, int n_q_heads, const int* err, cudaStream_t st);
 
-// Merge of the prefix chunks' statistics with the suffix result, per (sample, query head).
-cudaError_t launch_merge_prefix_suffix(const float* part, int n_chunks, int n_kv_heads, int rows_per_head,
-                                       const float* out_s, const float* lse_s, float* out, float* lse,
-                                       int n_samples, int n_q_heads, const int* err, cudaStream_t st);
-
 }  // namespace ta

@@ -1,0 +1,35 @@
+// Host-visible part of the short-unit decode kernel (short_decode.cu): its parameters and launcher.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace ta {
+
+constexpr int kShortMaxSeq = 128;       // sequences per launch
+constexpr int64_t kShortMaxLen = 2048;  // longest unit the automatic choice sends to this kernel
+
+// One launch: grid (KV heads, sequences), 128 threads, bf16 q/K/V with head_dim 128.
+struct ShortParams {
+  const __nv_bfloat16* q;  // [B][Hq][D], this launch's first sequence
+  const __nv_bfloat16* k;  // cache bases; kv_off[b] is relative to them
+  const __nv_bfloat16* v;
+  float* out;              // [B][Hq][D]
+  float* lse;              // [B][Hq]
+  const int* err;          // workspace error word (read when pre_part is set)
+  // Prefix chunk statistics folded into every row (nullptr: none); same layout as the split
+  // kernel's SplitParams::pre_part, already offset to this launch's first sequence.
+  const float* pre_part;
+  int pre_chunks, pre_rows, pre_stride;
+  int n_kv_heads, n_q_heads;
+  float scale_log2;
+  int64_t kv_off[kShortMaxSeq];   // element offset of sequence b's [Hkv][S_b][D] block
+  int64_t seq_len[kShortMaxSeq];
+};
+static_assert(sizeof(ShortParams) <= 4096, "kernel parameters must fit in 4 KB");
+
+// G = n_q_heads / n_kv_heads in {1, 2, 4, 8}.
+cudaError_t launch_short_decode(int G, int n_kv_heads, int batch, const ShortParams& p, cudaStream_t st);
+
+}  // namespace ta

@@ -72,6 +72,15 @@ struct SplitParams {
   int64_t bt_stride;
   int64_t num_pages;
   int32_t log2_page;
+  // Shared-prefix decode (bifurcated summary: the two parts' statistics merge exactly): the
+  // prefix pass's chunk statistics, folded into every row before it is written (nullptr: none).
+  // Row (sequence b of this launch, head g of KV head h) has pre_chunks entries at
+  // pre_part + ((c * n_kv_heads + h) * pre_rows + b * heads + g) * pre_stride, each m (log2
+  // units), l, two spare floats, o[D]; the pointer already skips the launch's earlier rows.
+  const float* pre_part;
+  int32_t pre_chunks;
+  int32_t pre_rows;
+  int32_t pre_stride;
   int64_t kv_off[kMaxSeqPerLaunch];
   int64_t seq_len[kMaxSeqPerLaunch];
   int64_t tile_off[kMaxSeqPerLaunch + 1];  // first tile of sequence b on the line
@@ -340,6 +349,27 @@ __device__ __forceinline__ float tree_sum(const float (&a)[M]) {
 // of another CTA propagate through the merge weights (2^(NaN - M) is NaN).
 __device__ __forceinline__ void write_final(const SplitParams& p, int b, int h, int r, int d, int D, float M,
                                             float L, float O, bool write_lse, bool poisoned) {
+  if (p.pre_part != nullptr) {
+    // The prefix chunks of this row, in chunk order: M' = max(M, m_c); L and O rescaled to M'.
+    const int64_t cstride = static_cast<int64_t>(p.n_kv_heads) * p.pre_rows * p.pre_stride;
+    const float* base =
+        p.pre_part + (static_cast<int64_t>(h) * p.pre_rows + (b << p.log2_heads) + r) * p.pre_stride;
+    float Mx = M;
+    for (int c = 0; c < p.pre_chunks; ++c) Mx = fmaxf(Mx, base[c * cstride]);
+    const float a = (M == -INFINITY) ? 0.f : ex2(M - Mx);
+    L *= a;
+    O *= a;
+    for (int c = 0; c < p.pre_chunks; ++c) {
+      const float* pc = base + c * cstride;
+      const float mc = pc[0];
+      const float w = (mc == -INFINITY) ? 0.f : ex2(mc - Mx);
+      L += w * pc[1];
+      O += w * pc[4 + d];
+    }
+    M = Mx;
+    // a prefix CTA that gave up left an empty partial and set the error word
+    poisoned = poisoned || *reinterpret_cast<const volatile int*>(p.err) != 0;
+  }
   float ov, lv;
   if (L > 0.f) {
     ov = O / L;

@@ -11,6 +11,7 @@
 
 #include "../../include/tree_attn.h"
 #include "bifurcated_tc.h"
+#include "short_decode.h"
 #include "split_kv_instances.h"
 
 namespace ta {
@@ -72,7 +73,7 @@ bool pick_kernel(ta_dtype dt, int D, int G, bool short_tiles, KernelInfo* ki, bo
 // shorter than 1024 tokens, unless the options force one.
 bool use_short_tiles(const int64_t* seqlens, int batch, const ta_options* opts) {
   if (opts && opts->split_tiles == 1) return false;
-  if (opts && opts->split_tiles == 2) return true;
+  if (opts && opts->split_tiles == 2) return true;  // (3, the short-unit kernel, only reaches suffix passes)
   int64_t total = 0;
   for (int b = 0; b < batch; ++b) total += seqlens[b];
   return batch > 0 && total < 1024LL * batch;
@@ -187,7 +188,7 @@ ta_status check_opts(const ta_options* o) {
   if (!o) return TA_OK;
   if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1) return TA_ERR_INVALID_ARG;
   if (o->prefix_path < 0 || o->prefix_path > 2) return TA_ERR_INVALID_ARG;
-  if (o->split_tiles < 0 || o->split_tiles > 2) return TA_ERR_INVALID_ARG;
+  if (o->split_tiles < 0 || o->split_tiles > 3) return TA_ERR_INVALID_ARG;
   for (int i = 0; i < 3; ++i)
     if (o->reserved[i] != 0) return TA_ERR_INVALID_ARG;
   return TA_OK;
@@ -234,10 +235,16 @@ struct PagedCache {
 
 // n_queries / q_first: query tokens per sequence and the first one this launch covers (the
 // kernel instance's G rows per unit are G / (Hq / Hkv) consecutive query tokens).
+// Prefix statistics folded into a suffix pass's final write (shared-prefix decode).
+struct PrefixFold {
+  const float* part = nullptr;  // [chunks][Hkv][rows][stride]
+  int chunks = 0, rows = 0, stride = 0;
+};
+
 ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, const void* k, const void* v,
                       float* out, float* lse, int Hq, int Hkv, int D, float scale, ta_dtype dt,
                       const ta_options* opts, uint8_t* body, int* err, cudaStream_t st, int n_queries = 1,
-                      int q_first = 0, const PagedCache* pc = nullptr) {
+                      int q_first = 0, const PagedCache* pc = nullptr, const PrefixFold* pf = nullptr) {
   const size_t qe = (dt == TA_BF16) ? 2 : 4;
   int log2_heads = 0;
   while ((1 << (log2_heads + 1)) <= Hq / Hkv) ++log2_heads;
@@ -267,6 +274,12 @@ ta_status launch_plan(const Plan& plan, const KernelInfo& ki, const void* q, con
     p.n_queries = n_queries;
     p.q_first = q_first;
     p.log2_heads = log2_heads;
+    if (pf) {
+      p.pre_part = pf->part + static_cast<int64_t>(g.b0) * (Hq / Hkv) * pf->stride;
+      p.pre_chunks = pf->chunks;
+      p.pre_rows = pf->rows;
+      p.pre_stride = pf->stride;
+    }
     if (pc) {
       p.block_table = pc->table + static_cast<int64_t>(g.b0) * pc->stride;
       p.bt_stride = pc->stride;
@@ -322,6 +335,22 @@ ta_status plan_for(const DecodeArgs& a, const ta_options* opts, const KernelInfo
   return build_plan(a.seqlens, a.kv_offsets, a.batch, a.Hkv, a.Hq / a.Hkv, a.D, ki.tile, slots, opts, plan);
 }
 
+// Plain bf16 decode with G = 8 query heads per KV head (head_dim 128) runs as the several-query
+// form with one query token: its G rows per (sequence, KV head) go to the tensor cores, which
+// read each K/V tile once for all of them (the split kernel's G = 8 instances are FP32-issue
+// bound).  ta_options.prefix_path 2 keeps the split kernel; 1 sends any bf16 head_dim-128 decode
+// to the tensor cores.
+bool decode_on_tensor_cores(const DecodeArgs& a, const ta_options* opts) {
+  if (a.dt != TA_BF16 || a.D != kBifD || a.kv_offsets != nullptr) return false;
+  const int path = opts ? opts->prefix_path : 0;
+  return path == 1 || (path == 0 && a.Hq / a.Hkv == 8);
+}
+
+// Decode through the several-query form (defined with it, below); with bytes_only it only
+// reports the workspace size.
+ta_status decode_tc(const DecodeArgs& a, const ta_options* opts, void* ws, size_t ws_bytes, cudaStream_t st,
+                    size_t* bytes_only);
+
 ta_status decode_with_workspace(const DecodeArgs& a, const ta_options* opts, void* ws, size_t ws_bytes,
                                 cudaStream_t st) {
   KernelInfo ki;
@@ -329,6 +358,7 @@ ta_status decode_with_workspace(const DecodeArgs& a, const ta_options* opts, voi
   ta_status s = validate(a, opts, true, &ki);
   if (s != TA_OK) return s;
   if (a.batch == 0) return TA_OK;
+  if (decode_on_tensor_cores(a, opts)) return decode_tc(a, opts, ws, ws_bytes, st, nullptr);
   if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
   s = plan_for(a, opts, ki, &plan);
   if (s != TA_OK) return s;
@@ -519,6 +549,18 @@ ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, 
   return TA_OK;
 }
 
+ta_status decode_tc(const DecodeArgs& a, const ta_options* opts, void* ws, size_t ws_bytes, cudaStream_t st,
+                    size_t* bytes_only) {
+  MultiPlan plan;
+  const ta_status s = multi_plan(a, 1, opts, &plan);
+  if (s != TA_OK) return s;
+  if (bytes_only) {
+    *bytes_only = kHeaderBytes + plan.body;
+    return TA_OK;
+  }
+  return multi_run(a, 1, opts, plan, ws, ws_bytes, st);
+}
+
 // ------------------------------------------------------------------------------------------
 // Bifurcated decode: prefix pass (all samples read the one shared prefix), suffix pass,
 // then an exact merge of the two softmax statistics per (sample, query head).
@@ -602,6 +644,7 @@ struct BifPlan {
   bool tc = false;
   int mtiles = 0, chunks = 0, rows_per_head = 0;
   size_t part_off = 0;
+  bool short_suffix = false;  // suffix pass on the short-unit kernel (tensor-core prefix pass only)
 };
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
@@ -714,6 +757,44 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
     bp->part_off = align_up(bp->total, kAlign);
     bp->total = bp->part_off +
                 sizeof(float) * static_cast<size_t>(chunks) * a.Hkv * bp->rows_per_head * kBifPartRow;
+    // Many short suffixes: one CTA per (sample, KV head) keeps every unit resident at once.
+    int64_t longest = 0;
+    for (int n = 0; n < a.N; ++n) longest = std::max(longest, a.suffix_lens[n]);
+    const int tiles_opt = opts ? opts->split_tiles : 0;
+    bp->short_suffix = tiles_opt == 3 ||
+                       (tiles_opt == 0 && static_cast<int64_t>(a.N) * a.Hkv >= sms && longest <= kShortMaxLen);
+  }
+  return TA_OK;
+}
+
+// The suffix pass on the short-unit kernel: one launch per 128 samples.
+ta_status launch_short(const BifArgs& a, const PrefixFold& pf, int* err, cudaStream_t st) {
+  const int G = a.Hq / a.Hkv;
+  int64_t off = 0;
+  for (int b0 = 0; b0 < a.N; b0 += kShortMaxSeq) {
+    const int nb = std::min(kShortMaxSeq, a.N - b0);
+    ShortParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.q = static_cast<const __nv_bfloat16*>(a.q) + static_cast<int64_t>(b0) * a.Hq * a.D;
+    sp.k = static_cast<const __nv_bfloat16*>(a.ks);
+    sp.v = static_cast<const __nv_bfloat16*>(a.vs);
+    sp.out = a.out + static_cast<int64_t>(b0) * a.Hq * a.D;
+    sp.lse = a.lse + static_cast<int64_t>(b0) * a.Hq;
+    sp.err = err;
+    sp.pre_part = pf.part + static_cast<int64_t>(b0) * G * pf.stride;
+    sp.pre_chunks = pf.chunks;
+    sp.pre_rows = pf.rows;
+    sp.pre_stride = pf.stride;
+    sp.n_kv_heads = a.Hkv;
+    sp.n_q_heads = a.Hq;
+    sp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
+    for (int i = 0; i < nb; ++i) {
+      sp.kv_off[i] = off;
+      sp.seq_len[i] = a.suffix_lens[b0 + i];
+      off += a.suffix_lens[b0 + i] * a.Hkv * a.D;
+    }
+    const cudaError_t e = launch_short_decode(G, a.Hkv, nb, sp, st);
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   return TA_OK;
 }
@@ -757,15 +838,20 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
       prof.end();
       const cudaEvent_t saved_start = g_prof_start, saved_stop = g_prof_stop;
       g_prof_start = g_prof_stop = nullptr;  // the suffix pass is not the main kernel here
-      s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, out_s, lse_s, a.Hq, a.Hkv, a.D, a.scale, TA_BF16, opts,
-                      base + bp.suffix_off, err, st);
+      // The suffix pass folds the prefix chunks' statistics into each row as it writes it.
+      PrefixFold pf;
+      pf.part = bpp.part;
+      pf.chunks = bp.chunks;
+      pf.rows = bp.rows_per_head;
+      pf.stride = kBifPartRow;
+      if (bp.short_suffix)
+        s = launch_short(a, pf, err, st);
+      else
+        s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, TA_BF16,
+                        opts, base + bp.suffix_off, err, st, 1, 0, nullptr, &pf);
       g_prof_start = saved_start;
       g_prof_stop = saved_stop;
-      if (s != TA_OK) return s;
-      e = launch_merge_prefix_suffix(bpp.part, bp.chunks, a.Hkv, bp.rows_per_head, out_s, lse_s, a.out, a.lse,
-                                     a.N, a.Hq, err, st);
-      if (e != cudaSuccess) return cuda_fail(e);
-      return TA_OK;
+      return s;
     }
     if (opts && opts->prefix_path == 1) return TA_ERR_UNSUPPORTED;
   }
@@ -820,6 +906,7 @@ ta_status tree_attn_workspace_size(const int64_t* seqlens, int32_t batch, int32_
   Plan plan;
   ta_status s = validate(a, opts, false, &ki);
   if (s != TA_OK) return s;
+  if (batch > 0 && decode_on_tensor_cores(a, opts)) return decode_tc(a, opts, nullptr, 0, nullptr, bytes);
   s = plan_for(a, opts, ki, &plan);
   if (s != TA_OK) return s;
   *bytes = kHeaderBytes + plan.body_bytes;
@@ -855,10 +942,16 @@ ta_status decode_alloc(const DecodeArgs& a, cudaStream_t st) {
   ta_status s = validate(a, nullptr, true, &ki);
   if (s != TA_OK) return s;
   if (a.batch == 0) return TA_OK;
-  s = plan_for(a, nullptr, ki, &plan);
+  size_t bytes = 0;
+  if (decode_on_tensor_cores(a, nullptr)) {
+    s = decode_tc(a, nullptr, nullptr, 0, st, &bytes);
+  } else {
+    s = plan_for(a, nullptr, ki, &plan);
+    bytes = kHeaderBytes + plan.body_bytes;
+  }
   if (s != TA_OK) return s;
   PlainCtx ctx{a};
-  return with_temp_workspace(kHeaderBytes + plan.body_bytes, st, &plain_run, &ctx);
+  return with_temp_workspace(bytes, st, &plain_run, &ctx);
 }
 }  // namespace
 

@@ -82,14 +82,20 @@ typedef struct {
   int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
                               consumers' wait runs out (no fault: the data simply never arrives).
                               Tensor-core passes: CTA (0, 0, 0) never loads this K tile */
-  int32_t prefix_path;     /* bifurcated and multi-query calls.  Bifurcated: 0 automatic (tensor-
-                              core prefix pass when head_dim is 128 and the prefix is not empty);
-                              1 tensor-core pass (TA_ERR_UNSUPPORTED if not possible); 2 split-KV
-                              pass per sample.  Multi-query: 0 automatic (tensor cores when bf16,
-                              head_dim 128 and 8 <= G * n <= 128); 1 tensor cores; 2 split-KV
-                              passes */
+  int32_t prefix_path;     /* bifurcated, multi-query and decode calls.  Bifurcated: 0 automatic
+                              (tensor-core prefix pass when head_dim is 128 and the prefix is not
+                              empty); 1 tensor-core pass (TA_ERR_UNSUPPORTED if not possible); 2
+                              split-KV pass per sample.  Multi-query: 0 automatic (tensor cores
+                              when bf16, head_dim 128 and 8 <= G * n <= 128); 1 tensor cores; 2
+                              split-KV passes.  Decode (tree_attn_decode_ex / _decode, bf16, head_dim
+                              128): 0 automatic (tensor cores when G = 8, the split kernel otherwise);
+                              1 tensor cores; 2 split kernel */
   int32_t split_tiles;     /* split-KV tile configuration.  0: automatic (short tiles when the mean
-                              sequence is under 1024 tokens); 1: long tiles; 2: short tiles */
+                              sequence is under 1024 tokens); 1: long tiles; 2: short tiles.
+                              Shared-prefix calls with the tensor-core prefix pass: the suffix pass
+                              runs on the short-unit kernel (one CTA per sample and KV head) when
+                              head_dim is 128, there are at least as many (sample, KV head) units as
+                              SMs and no suffix exceeds 2048 tokens, or always with 3 */
   int32_t reserved[3];     /* must be 0 */
 } ta_options;
 
@@ -154,7 +160,10 @@ ta_status tree_attn_decode_f32(const float* q, const float* k_cache, const float
  * Decode attention with a caller-owned workspace (no allocation; one kernel
  * launch per 128 sequences).  `workspace` must be 256-byte aligned, at least
  * tree_attn_workspace_size() bytes, zero-filled before first use, and not used
- * by two calls in flight at once.  `opts` may be NULL.
+ * by two calls in flight at once.  `opts` may be NULL.  bf16 calls with head_dim
+ * 128 and G = 8 query heads per KV head run on the tensor cores (the several-query
+ * form of tree_attn_decode_multi_ex with one query token: a tcgen05 launch and a
+ * merge launch per 128 sequences); ta_options.prefix_path selects the path.
  */
 ta_status tree_attn_decode_ex(ta_dtype dtype, const void* q, const void* k_cache, const void* v_cache,
                               const int64_t* seqlens, int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,

@@ -9,7 +9,7 @@ from gpu_util import compare, device_tensor, empty_outputs, new_workspace
 pytestmark = pytest.mark.gpu
 
 
-def bif_gpu(inp, sp, entry="ex", prefix_path=0):
+def bif_gpu(inp, sp, entry="ex", prefix_path=0, split_tiles=0):
     import torch
 
     import exact_long_context_split_b200 as ta
@@ -21,7 +21,7 @@ def bif_gpu(inp, sp, entry="ex", prefix_path=0):
     out, lse = empty_outputs(N, Hq, D)
     lens = [int(s) for s in sp.suffix_lens]
     if entry == "ex":
-        opts = ta.make_options(prefix_path=prefix_path)
+        opts = ta.make_options(prefix_path=prefix_path, split_tiles=split_tiles)
         ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(P, lens, Hq, Hkv, D, opts))
         ta.tree_attn_decode_bifurcated_ex(q, kp, vp, P, ks, vs, lens, Hq, Hkv, D, sp.scale, out, lse, opts, ws)
         assert ta.tree_attn_check(ws) == ta.TA_OK
@@ -76,6 +76,28 @@ def test_bifurcated_prefix_paths(prefix_len, suffix_lens, Hq, Hkv, D, prefix_pat
     compare(out, lse, *oracle_bif(inp, sp))
 
 
+# The suffix pass on the short-unit kernel (one CTA per sample and KV head, the prefix chunks'
+# statistics folded into each row): ragged suffixes with empty and one-token ones, every G, more
+# than 128 samples (two launches).
+SHORT_CASES = [
+    (1000, [0, 1, 31, 32, 33, 300, 2047, 5], 32, 8, 128),
+    (65, [3, 70], 8, 2, 128),
+    (300, [9] * 64, 16, 2, 128),
+    (64, [0, 2, 128], 8, 8, 128),
+    (4097, [100] * 140, 16, 8, 128),
+]
+
+
+@pytest.mark.parametrize("prefix_len,suffix_lens,Hq,Hkv,D", SHORT_CASES)
+def test_short_unit_suffix_pass(prefix_len, suffix_lens, Hq, Hkv, D):
+    sp = synth.BifurcatedSpec("case", prefix_len, suffix_lens, Hq, Hkv, D, seed=25)
+    inp = synth.make_bifurcated_inputs(sp)
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path=1, split_tiles=3)
+    compare(out, lse, *oracle_bif(inp, sp))
+    again = bif_gpu(inp, sp, "ex", prefix_path=1, split_tiles=3)
+    assert np.array_equal(out.view(np.uint32), again[0].view(np.uint32))
+
+
 def test_tensor_core_prefix_is_deterministic():
     sp = synth.BifurcatedSpec("case", 20000, [50] * 32, 32, 8, 128, seed=24)
     inp = synth.make_bifurcated_inputs(sp)
@@ -120,15 +142,16 @@ def test_bifurcated_equals_plain_decode_of_concatenation():
     compare(out, lse, plain_out.astype(np.float64), plain_lse.astype(np.float64))
 
 
-@pytest.mark.parametrize("prefix_path", [1, 2])
-def test_bifurcated_config_sampled(prefix_path):
-    """The shared-prefix workload (64 samples, 65,536 + 256 tokens): every query head of 16
-    samples spread over the batch."""
+@pytest.mark.parametrize("prefix_path,split_tiles", [(1, 0), (1, 1), (2, 0)])
+def test_bifurcated_config_sampled(prefix_path, split_tiles):
+    """The shared-prefix workload (64 samples, 65,536 + 256 tokens): every query head of 17
+    samples spread over the batch; the suffix pass on the short-unit kernel (automatic), on the
+    split kernel (split_tiles 1), and the all-split path (prefix_path 2)."""
     from gpu_util import oracle_parallel
 
     sp = synth.bifurcated_configs()["shared_prefix"]
     inp = synth.make_bifurcated_inputs(sp)
-    out, lse = bif_gpu(inp, sp, "ex", prefix_path)
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path, split_tiles)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
     samples = list(range(0, sp.n_samples, 4)) + [sp.n_samples - 1]
     tasks = [[(n, h) for h in range(sp.n_q_heads)] for n in samples]

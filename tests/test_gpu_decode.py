@@ -37,9 +37,40 @@ def test_every_instance_ragged(dtype, D, G, tiles):
     Hkv = 2
     sp = spec(RAGGED, G * Hkv, Hkv, D, dtype=dtype, seed=100 + G + D)
     inp = synth.make_decode_inputs(sp)
-    out, lse = decode_gpu(inp, sp, ta.make_options(split_tiles=tiles))
+    out, lse = decode_gpu(inp, sp, ta.make_options(split_tiles=tiles, prefix_path=ta.PREFIX_SPLIT_KV))
     ref_out, ref_lse = oracle_of(inp, sp)
     compare(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (64, 8), (8, 1)])
+def test_g8_decode_on_tensor_cores(Hq, Hkv):
+    """G = 8 bf16 decode (head_dim 128) runs on the tensor cores by default: ragged lengths with
+    an empty and a one-token sequence against the oracle, bit-identical across runs, and within
+    the tolerance of the split kernel (prefix_path 2)."""
+    import exact_long_context_split_b200 as ta
+
+    sp = spec([1, 0, 129, 1000, 20000], Hq, Hkv, 128, seed=14, spike_frac=0.001)
+    inp = synth.make_decode_inputs(sp)
+    out, lse = decode_gpu(inp, sp)
+    ref_out, ref_lse = oracle_of(inp, sp)
+    compare(out, lse, ref_out, ref_lse)
+    out2, lse2 = decode_gpu(inp, sp)
+    assert np.array_equal(out.view(np.uint32), out2.view(np.uint32))
+    assert np.array_equal(lse.view(np.uint32), lse2.view(np.uint32))
+    s_out, s_lse = decode_gpu(inp, sp, ta.make_options(prefix_path=ta.PREFIX_SPLIT_KV))
+    compare(s_out, s_lse, ref_out, ref_lse)
+    a_out, a_lse = decode_gpu(inp, sp, entry="alloc")
+    assert np.array_equal(out.view(np.uint32), a_out.view(np.uint32))
+
+
+def test_tensor_core_decode_forced_for_g4():
+    """prefix_path 1 sends G = 4 bf16 decode to the tensor cores as well."""
+    import exact_long_context_split_b200 as ta
+
+    sp = spec([3000, 5, 0], 32, 8, 128, seed=15)
+    inp = synth.make_decode_inputs(sp)
+    out, lse = decode_gpu(inp, sp, ta.make_options(prefix_path=ta.PREFIX_TENSOR_CORE))
+    compare(out, lse, *oracle_of(inp, sp))
 
 
 @pytest.mark.parametrize("tiles", [1, 2])
