@@ -33,6 +33,12 @@ constexpr float kShortRescale = 8.0f;
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Ask the TMA engine to bring [src, src + bytes) into L2 (16-byte aligned, a multiple of 16
+// bytes); nothing is written to shared memory and no barrier is involved.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
@@ -56,6 +62,17 @@ __global__ void __launch_bounds__(kWarps * 32, 4) short_decode_kernel(const __gr
   const __nv_bfloat16* V = p.v + p.kv_off[b] + static_cast<int64_t>(h) * S * kD;
   const int64_t qrow0 = static_cast<int64_t>(b) * p.n_q_heads + h * G;  // first output row of the unit
 
+  // The whole unit's K and V (S rows of 256 bytes each) are requested into L2 at once, so every
+  // unit resident on the GPU streams from HBM together; the warps' loads then find L2.
+  if (warp == 0) {
+    constexpr int64_t kPiece = 64 * 1024;
+    const int64_t bytes = S * kD * 2;
+    for (int64_t off = lane * kPiece; off < bytes; off += 32 * kPiece) {
+      const uint32_t n = static_cast<uint32_t>(min(kPiece, bytes - off));
+      prefetch_l2(reinterpret_cast<const uint8_t*>(K) + off, n);
+      prefetch_l2(reinterpret_cast<const uint8_t*>(V) + off, n);
+    }
+  }
   for (int i = tid; i < G * kD; i += kWarps * 32)
     qs[i / kD][i % kD] = __bfloat162float(p.q[qrow0 * kD + i]) * p.scale_log2;
   __syncthreads();
@@ -149,41 +166,81 @@ __global__ void __launch_bounds__(kWarps * 32, 4) short_decode_kernel(const __gr
     *reinterpret_cast<float4*>(&wo[warp][g][4 * lane]) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
   }
   __syncthreads();
-  // merge the warps in order, fold in the prefix chunks, write out = o / l and lse
-  const bool prefix_failed = p.pre_part != nullptr && *reinterpret_cast<const volatile int*>(p.err) != 0;
-  for (int i = tid; i < G * kD; i += kWarps * 32) {
-    const int g = i / kD, d = i % kD;
+  // merge the warps in order, fold in the prefix chunks, write out = o / l and lse.  The row
+  // statistics first (one thread per row: the max over warps and chunks, the weights, l), then
+  // every thread a float4 of columns with all of its chunk loads independent.
+  __shared__ float rM[G], rL[G], rw[G][kWarps];
+  __shared__ float cm[G][kShortMaxChunks], cw[G][kShortMaxChunks];  // chunk m, then its weight
+  __shared__ float cl[G][kShortMaxChunks];
+  const bool fold = p.pre_part != nullptr;
+  const int nc = fold ? p.pre_chunks : 0;
+  const int64_t cstride = static_cast<int64_t>(p.n_kv_heads) * p.pre_rows * p.pre_stride;
+  auto chunk_row = [&](int g) {
+    return p.pre_part + (static_cast<int64_t>(h) * p.pre_rows + b * G + g) * p.pre_stride;
+  };
+  for (int i = tid; i < G * nc; i += kWarps * 32) {  // every chunk's (m, l) of every row at once
+    const int g = i / nc, c = i % nc;
+    const float* pc = chunk_row(g) + c * cstride;
+    cm[g][c] = pc[0];
+    cl[g][c] = pc[1];
+  }
+  __syncthreads();
+  if (tid < G) {
+    const int g = tid;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w][g]);
-    const float* pre = nullptr;
-    int64_t cstride = 0;
-    if (p.pre_part != nullptr) {
-      cstride = static_cast<int64_t>(p.n_kv_heads) * p.pre_rows * p.pre_stride;
-      pre = p.pre_part + (static_cast<int64_t>(h) * p.pre_rows + b * G + g) * p.pre_stride;
-      for (int c = 0; c < p.pre_chunks; ++c) M = fmaxf(M, pre[c * cstride]);
-    }
-    float L = 0.f, O = 0.f;
+    for (int c = 0; c < nc; ++c) M = fmaxf(M, cm[g][c]);
+    float L = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       const float a = (wm[w][g] == -INFINITY) ? 0.f : ex2(wm[w][g] - M);
+      rw[g][w] = a;
       L += a * wl[w][g];
-      O += a * wo[w][g][d];
     }
-    for (int c = 0; pre != nullptr && c < p.pre_chunks; ++c) {
-      const float* pc = pre + c * cstride;
-      const float a = (pc[0] == -INFINITY) ? 0.f : ex2(pc[0] - M);
-      L += a * pc[1];
-      O += a * pc[4 + d];
+    for (int c = 0; c < nc; ++c) {
+      const float a = (cm[g][c] == -INFINITY) ? 0.f : ex2(cm[g][c] - M);
+      cw[g][c] = a;
+      L += a * cl[g][c];
     }
-    float ov = 0.f, lv = -INFINITY;
+    rM[g] = M;
+    rL[g] = L;
+  }
+  __syncthreads();
+  const bool prefix_failed = fold && *reinterpret_cast<const volatile int*>(p.err) != 0;
+  for (int i = tid; i < G * (kD / 4); i += kWarps * 32) {
+    const int g = i / (kD / 4), d4 = (i % (kD / 4)) * 4;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float a = rw[g][w];
+      const float4 o = *reinterpret_cast<const float4*>(&wo[w][g][d4]);
+      O = make_float4(O.x + a * o.x, O.y + a * o.y, O.z + a * o.z, O.w + a * o.w);
+    }
+    if (fold) {
+      const float* pre = chunk_row(g) + 4 + d4;
+#pragma unroll 6
+      for (int c = 0; c < p.pre_chunks; ++c) {
+        const float a = cw[g][c];
+        const float4 o = *reinterpret_cast<const float4*>(pre + c * cstride);
+        O = make_float4(O.x + a * o.x, O.y + a * o.y, O.z + a * o.z, O.w + a * o.w);
+      }
+    }
+    const float L = rL[g];
+    float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lv = -INFINITY;
     if (L > 0.f) {
-      ov = O / L;
-      lv = (M + log2f(L)) * 0.693147180559945309f;
+      const float inv = 1.f / L;
+      ov = make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+      lv = (rM[g] + log2f(L)) * 0.693147180559945309f;
     }
-    if (prefix_failed || L != L) ov = lv = __int_as_float(0x7fc00000);
-    p.out[(qrow0 + g) * kD + d] = ov;
-    if (d == 0) p.lse[qrow0 + g] = lv;
+    if (prefix_failed || L != L) {
+      const float nan = __int_as_float(0x7fc00000);
+      ov = make_float4(nan, nan, nan, nan);
+      lv = nan;
+    }
+    *reinterpret_cast<float4*>(p.out + (qrow0 + g) * kD + d4) = ov;
+    if (d4 == 0) p.lse[qrow0 + g] = lv;
   }
 }
 

@@ -9,6 +9,7 @@ namespace ta {
 
 constexpr int kShortMaxSeq = 128;       // sequences per launch
 constexpr int64_t kShortMaxLen = 2048;  // longest unit the automatic choice sends to this kernel
+constexpr int kShortMaxChunks = 64;     // prefix chunks it can fold per row
 
 // One launch: grid (KV heads, sequences), 128 threads, bf16 q/K/V with head_dim 128.
 struct ShortParams {

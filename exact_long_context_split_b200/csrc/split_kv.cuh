@@ -355,10 +355,12 @@ __device__ __forceinline__ void write_final(const SplitParams& p, int b, int h, 
     const float* base =
         p.pre_part + (static_cast<int64_t>(h) * p.pre_rows + (b << p.log2_heads) + r) * p.pre_stride;
     float Mx = M;
+#pragma unroll 6
     for (int c = 0; c < p.pre_chunks; ++c) Mx = fmaxf(Mx, base[c * cstride]);
     const float a = (M == -INFINITY) ? 0.f : ex2(M - Mx);
     L *= a;
     O *= a;
+#pragma unroll 6
     for (int c = 0; c < p.pre_chunks; ++c) {
       const float* pc = base + c * cstride;
       const float mc = pc[0];

@@ -761,8 +761,9 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
     int64_t longest = 0;
     for (int n = 0; n < a.N; ++n) longest = std::max(longest, a.suffix_lens[n]);
     const int tiles_opt = opts ? opts->split_tiles : 0;
-    bp->short_suffix = tiles_opt == 3 ||
-                       (tiles_opt == 0 && static_cast<int64_t>(a.N) * a.Hkv >= sms && longest <= kShortMaxLen);
+    bp->short_suffix = a.D == 128 && chunks <= kShortMaxChunks &&
+                       (tiles_opt == 3 ||
+                        (tiles_opt == 0 && static_cast<int64_t>(a.N) * a.Hkv >= sms && longest <= kShortMaxLen));
   }
   return TA_OK;
 }
