@@ -76,7 +76,8 @@ typedef enum { TA_BF16 = 0, TA_F32 = 1 } ta_dtype;
 
 /* Optional tuning and test hooks; pass NULL for the defaults (all fields 0 / -1). */
 typedef struct {
-  int32_t num_ctas;        /* 0: one CTA per resident slot (SMs x CTAs per SM); else the split grid size */
+  int32_t num_ctas;        /* 0: one CTA per resident slot (SMs x CTAs per SM), at most one per two
+                              tiles; else the split grid size */
   int32_t wait_limit_us;   /* 0: 2,000,000 us.  Bound on every wait inside a kernel; on expiry the
                               kernel records TA_ERR_TIMEOUT in the workspace and returns */
   int32_t debug_skip_tile; /* -1: off.  Test hook: CTA 0 never loads this tile of its range, so its
