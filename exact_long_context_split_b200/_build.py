@@ -54,13 +54,15 @@ def _deps(path: str, seen=None) -> set:
 
 
 def _hash_files(paths, extra=()) -> str:
+    """Hash of the files (by path relative to the repository root) and of the flags, with the
+    include directory written relative too: the same tree gives the same hash wherever it sits."""
     h = hashlib.sha256()
-    for f in sorted(paths):
+    for f in sorted(paths, key=lambda f: os.path.relpath(f, ROOT)):
         h.update(os.path.relpath(f, ROOT).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
     for x in extra:
-        h.update(x.encode())
+        h.update((os.path.relpath(x, ROOT) if os.path.isabs(x) else x).encode())
     return h.hexdigest()[:32]
 
 

@@ -9,8 +9,7 @@
 // attention").
 //
 // Per warp, per chunk of 32 keys (online softmax of the "Attention acceleration" concept page,
-// compassingai.com, Technical principles 2.1, in base 2, O kept unnormalised), with the chunk's
-// K and V loads all in flight together (one memory round trip per chunk):
+// compassingai.com, Technical principles 2.1, in base 2, O kept unnormalised):
 //   scores:  lane j holds key c0 + j: x_g = (q_g s log2 e) . k for the G query heads of the unit
 //   softmax: chunk max per head (warp shuffles); the running max m_g moves only when the chunk's
 //            exceeds it by more than 8 (lazy rescale: exact, l and o share the reference)
@@ -34,12 +33,6 @@ constexpr float kShortRescale = 8.0f;
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Ask the TMA engine to bring [src, src + bytes) into L2 (16-byte aligned, a multiple of 16
-// bytes); nothing is written to shared memory and no barrier is involved.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
@@ -52,7 +45,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int G>
-__global__ void __launch_bounds__(kWarps * 32, 2) short_decode_kernel(const __grid_constant__ ShortParams p) {
+__global__ void __launch_bounds__(kWarps * 32, 4) short_decode_kernel(const __grid_constant__ ShortParams p) {
   __shared__ __align__(16) float qs[G][kD];  // q * scale * log2(e)
   __shared__ float wm[kWarps][G], wl[kWarps][G];
   __shared__ __align__(16) float wo[kWarps][G][kD];
@@ -63,17 +56,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) short_decode_kernel(const __gr
   const __nv_bfloat16* V = p.v + p.kv_off[b] + static_cast<int64_t>(h) * S * kD;
   const int64_t qrow0 = static_cast<int64_t>(b) * p.n_q_heads + h * G;  // first output row of the unit
 
-  // The whole unit's K and V (S rows of 256 bytes each) are requested into L2 at once, so every
-  // unit resident on the GPU streams from HBM together; the warps' loads then find L2.
-  if (warp == 0) {
-    constexpr int64_t kPiece = 64 * 1024;
-    const int64_t bytes = S * kD * 2;
-    for (int64_t off = lane * kPiece; off < bytes; off += 32 * kPiece) {
-      const uint32_t n = static_cast<uint32_t>(min(kPiece, bytes - off));
-      prefetch_l2(reinterpret_cast<const uint8_t*>(K) + off, n);
-      prefetch_l2(reinterpret_cast<const uint8_t*>(V) + off, n);
-    }
-  }
   for (int i = tid; i < G * kD; i += kWarps * 32)
     qs[i / kD][i % kD] = __bfloat162float(p.q[qrow0 * kD + i]) * p.scale_log2;
   __syncthreads();
@@ -90,36 +72,37 @@ __global__ void __launch_bounds__(kWarps * 32, 2) short_decode_kernel(const __gr
   for (int64_t c0 = t0; c0 < t1; c0 += 32) {
     const int nk = static_cast<int>(min(static_cast<int64_t>(32), t1 - c0));
     const bool valid = lane < nk;
-    // One memory round trip per chunk: the lane's whole key row (16 x 16 bytes) and its four
-    // columns of all 32 value rows (32 x 8 bytes) are requested together.
-    uint4 kr[kD / 8];
+    // scores: the lane's key row in two halves of 128 bytes, each half's 8 loads in flight together
     const uint4* krow = reinterpret_cast<const uint4*>(K + (c0 + lane) * kD);
+    float s0[G], s1[G];
 #pragma unroll
-    for (int e = 0; e < kD / 8; ++e) kr[e] = valid ? __ldg(krow + e) : make_uint4(0, 0, 0, 0);
-    uint2 vr[32];
-    const uint2* vcol = reinterpret_cast<const uint2*>(V + c0 * kD) + lane;
+    for (int g = 0; g < G; ++g) s0[g] = s1[g] = 0.f;
 #pragma unroll
-    for (int u = 0; u < 32; ++u) vr[u] = (u < nk) ? __ldg(vcol + u * (kD / 4)) : make_uint2(0, 0);
-    // scores: x_g = (q_g s log2 e) . k for the lane's key
+    for (int half = 0; half < 2; ++half) {
+      uint4 kr[kD / 16];
+#pragma unroll
+      for (int e = 0; e < kD / 16; ++e) kr[e] = valid ? __ldg(krow + half * (kD / 16) + e) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+#pragma unroll
+        for (int e = 0; e < kD / 16; ++e) {
+          const int c = 8 * (half * (kD / 16) + e);  // first column of chunk e
+          const float4 qa = *reinterpret_cast<const float4*>(&qs[g][c]);
+          const float4 qb = *reinterpret_cast<const float4*>(&qs[g][c + 4]);
+          s0[g] = fmaf(qa.x, bf_lo(kr[e].x), s0[g]);
+          s1[g] = fmaf(qa.y, bf_hi(kr[e].x), s1[g]);
+          s0[g] = fmaf(qa.z, bf_lo(kr[e].y), s0[g]);
+          s1[g] = fmaf(qa.w, bf_hi(kr[e].y), s1[g]);
+          s0[g] = fmaf(qb.x, bf_lo(kr[e].z), s0[g]);
+          s1[g] = fmaf(qb.y, bf_hi(kr[e].z), s1[g]);
+          s0[g] = fmaf(qb.z, bf_lo(kr[e].w), s0[g]);
+          s1[g] = fmaf(qb.w, bf_hi(kr[e].w), s1[g]);
+        }
+      }
+    }
     float x[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int e = 0; e < kD / 8; ++e) {
-        const float4 qa = *reinterpret_cast<const float4*>(&qs[g][8 * e]);
-        const float4 qb = *reinterpret_cast<const float4*>(&qs[g][8 * e + 4]);
-        s0 = fmaf(qa.x, bf_lo(kr[e].x), s0);
-        s1 = fmaf(qa.y, bf_hi(kr[e].x), s1);
-        s0 = fmaf(qa.z, bf_lo(kr[e].y), s0);
-        s1 = fmaf(qa.w, bf_hi(kr[e].y), s1);
-        s0 = fmaf(qb.x, bf_lo(kr[e].z), s0);
-        s1 = fmaf(qb.y, bf_hi(kr[e].z), s1);
-        s0 = fmaf(qb.z, bf_lo(kr[e].w), s0);
-        s1 = fmaf(qb.w, bf_hi(kr[e].w), s1);
-      }
-      x[g] = valid ? s0 + s1 : -INFINITY;
-    }
+    for (int g = 0; g < G; ++g) x[g] = valid ? s0[g] + s1[g] : -INFINITY;
     // online softmax (base 2), lazy rescale
     float pg[G];
 #pragma unroll
@@ -135,17 +118,23 @@ __global__ void __launch_bounds__(kWarps * 32, 2) short_decode_kernel(const __gr
       pg[g] = valid ? ex2(x[g] - m[g]) : 0.f;
       lp[g] += pg[g];
     }
-    // p V: lane j owns columns 4 j .. 4 j + 3; key u's weight comes from lane u (0 past nk)
+    // p V: lane j owns columns 4 j .. 4 j + 3; V rows loaded 8 at a time
+    const uint2* vcol = reinterpret_cast<const uint2*>(V + c0 * kD) + lane;
+    for (int j0 = 0; j0 < nk; j0 += 8) {
+      uint2 vr[8];
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const float v0 = bf_lo(vr[u].x), v1 = bf_hi(vr[u].x), v2 = bf_lo(vr[u].y), v3 = bf_hi(vr[u].y);
+      for (int u = 0; u < 8; ++u) vr[u] = (j0 + u < nk) ? __ldg(vcol + (j0 + u) * (kD / 4)) : make_uint2(0, 0);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float w = __shfl_sync(0xffffffffu, pg[g], u);
-        acc[g][0] = fmaf(w, v0, acc[g][0]);
-        acc[g][1] = fmaf(w, v1, acc[g][1]);
-        acc[g][2] = fmaf(w, v2, acc[g][2]);
-        acc[g][3] = fmaf(w, v3, acc[g][3]);
+      for (int u = 0; u < 8; ++u) {
+        const float v0 = bf_lo(vr[u].x), v1 = bf_hi(vr[u].x), v2 = bf_lo(vr[u].y), v3 = bf_hi(vr[u].y);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float w = __shfl_sync(0xffffffffu, pg[g], j0 + u);  // 0 past the chunk's keys
+          acc[g][0] = fmaf(w, v0, acc[g][0]);
+          acc[g][1] = fmaf(w, v1, acc[g][1]);
+          acc[g][2] = fmaf(w, v2, acc[g][2]);
+          acc[g][3] = fmaf(w, v3, acc[g][3]);
+        }
       }
     }
   }

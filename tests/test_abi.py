@@ -121,3 +121,21 @@ def test_workspace_entry_points_validate():
     sz = ctypes.c_size_t(0)
     assert L.tree_attn_workspace_size(arr, 1, 6, 4, 128, 0, None, ctypes.byref(sz)) == ta.TA_ERR_INVALID_ARG
     assert L.tree_attn_workspace_size(arr, 1, 4, 4, 128, 0, None, None) == ta.TA_ERR_INVALID_ARG
+
+
+def test_build_id_does_not_depend_on_where_the_tree_sits(tmp_path):
+    """The library carries a hash of its sources; a copy of the tree at another absolute path
+    (as on a GPU machine) must hash the same, or the loaded library would be refused there."""
+    import shutil
+    import subprocess
+    import sys
+
+    shutil.copytree(os.path.join(ROOT, "exact_long_context_split_b200"), tmp_path / "exact_long_context_split_b200",
+                    ignore=shutil.ignore_patterns("_build", "*.so", "*.hash", "__pycache__"))
+    shutil.copytree(os.path.join(ROOT, "include"), tmp_path / "include")
+    code = "import sys; sys.path.insert(0, sys.argv[1]); from exact_long_context_split_b200 import _build; " \
+           "print(_build.source_hash())"
+    there = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, check=True)
+    from exact_long_context_split_b200 import _build
+
+    assert there.stdout.strip() == _build.source_hash() == ta.tree_attn_build_id()
