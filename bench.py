@@ -383,6 +383,9 @@ class DecodeRun:
         self.tokens = spec.tokens
         self.flops = 4 * D * Hq * sum(self.seqlens)
         self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv},{'ShortTiles' if sum(self.seqlens) < 1024 * len(self.seqlens) else 'LongTiles'}>"
+        if D == 128 and Hq // Hkv == 8:  # bf16 decode with G = 8 runs on the tensor cores
+            self.launches_per_step = 2 * ((B + 127) // 128)
+            self.kernel = "bif_prefix_kernel (decode, 8 rows per KV head)"
 
     def step(self, stream):
         sp = self.spec
@@ -490,10 +493,11 @@ class PagedMultiRun(PagedRun):
 
 
 class BifurcatedRun:
-    """Shared-prefix workload: one call = the tensor-core prefix pass, the suffix pass and the
-    exact merge.  The roofline is the prefix pass's dense contraction on the tensor cores."""
+    """Shared-prefix workload: one call = the tensor-core prefix pass and the suffix pass, which
+    folds the prefix chunks' statistics into each row as it writes it (two launches per group of
+    128 samples).  The roofline is the prefix pass's dense contraction on the tensor cores."""
 
-    launches_per_step = 3
+    launches_per_step = 2
     metric, unit, bound = METRIC, UNIT, "tensor"
     inputs = None
 
@@ -513,6 +517,7 @@ class BifurcatedRun:
         ta.tree_attn_workspace_init(self.ws)
         self.kv_bytes = spec.kv_bytes
         self.tokens = spec.prefix_len + sum(self.lens)
+        self.launches_per_step = 2 * ((N + 127) // 128)
         self.flops = 4 * D * N * Hq * spec.prefix_len  # the prefix pass: S = Q K^T and O = P V
         self.kernel = "bif_prefix_kernel (shared-prefix pass; the step adds the suffix pass and the merge)"
 

@@ -161,3 +161,89 @@ def test_tensor_core_multi_query_bounded_wait_runs_out():
     ref_out, ref_lse = oracle.multi_query_attention(inp["q"], inp["k"], inp["v"], lens, 4, 32, 8, 128, sp.scale)
     compare(out.cpu().numpy().reshape(8, 32, 128), lse.cpu().numpy().reshape(8, 32),
             ref_out.reshape(8, 32, 128), ref_lse.reshape(8, 32))
+
+
+def test_shared_prefix_bounded_wait_runs_out():
+    """The hook in the shared-prefix tensor-core pass (two M tiles per CTA): CTA (0, 0, 0) never
+    loads K tile 0, its waits run out, the suffix pass sees the error word and writes NaN for
+    every row; after re-initialising the workspace the same call is exact."""
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    sp = synth.BifurcatedSpec("case", 3000, [5, 0, 300, 40], 32, 8, 128, seed=45)
+    inp = synth.make_bifurcated_inputs(sp)
+    q, kp, vp, ks, vs = (device_tensor(inp[n], "bf16") for n in ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix"))
+    lens = [int(s) for s in sp.suffix_lens]
+    out = torch.empty(4, 32, 128, device="cuda")
+    lse = torch.empty(4, 32, device="cuda")
+    for opts, expect in ((ta.make_options(wait_limit_us=20000, debug_skip_tile=0, prefix_path=1, split_tiles=3),
+                          ta.TA_ERR_TIMEOUT),
+                         (ta.make_options(prefix_path=1, split_tiles=3), ta.TA_OK)):
+        ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(3000, lens, 32, 8, 128, opts))
+        ta.tree_attn_decode_bifurcated_ex(q, kp, vp, 3000, ks, vs, lens, 32, 8, 128, sp.scale, out, lse, opts, ws)
+        assert ta.tree_attn_check(ws) == expect
+        if expect == ta.TA_ERR_TIMEOUT:
+            assert torch.isnan(out).all() and torch.isnan(lse).all()
+    ref = oracle.bifurcated_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], 3000, inp["k_suffix"],
+                                      inp["v_suffix"], lens, 32, 8, 128, sp.scale)
+    compare(out.cpu().numpy(), lse.cpu().numpy(), *ref)
+
+
+@pytest.mark.parametrize("call", ["decode", "g8_decode", "bifurcated", "anchor"])
+def test_profile_events_bracket_the_main_kernel(call):
+    """tree_attn_profile_events: the library records the events on the call's stream around its
+    main kernel; the span lies inside the whole call's span, and turning the hook off stops the
+    recording."""
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    inner = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for e in inner:
+        e.record()  # torch creates the CUDA event on its first record
+    torch.cuda.synchronize()
+    if call in ("decode", "g8_decode"):
+        Hq = 32 if call == "decode" else 64
+        sp = synth.DecodeSpec("p", [20000, 3000], Hq, 8, 128, seed=46)
+        inp = synth.make_decode_inputs(sp)
+        q, k, v = (device_tensor(inp[n], "bf16") for n in ("q", "k", "v"))
+        out, lse = torch.empty(2, Hq, 128, device="cuda"), torch.empty(2, Hq, device="cuda")
+        ws = new_workspace(ta.tree_attn_workspace_size([20000, 3000], Hq, 8, 128))
+        run = lambda: ta.tree_attn_decode_ex("bf16", q, k, v, [20000, 3000], Hq, 8, 128, sp.scale, out, lse,  # noqa: E731
+                                             None, ws)
+    elif call == "bifurcated":
+        sp = synth.BifurcatedSpec("p", 5000, [100] * 40, 32, 8, 128, seed=47)
+        inp = synth.make_bifurcated_inputs(sp)
+        d = {n: device_tensor(inp[n], "bf16") for n in ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix")}
+        out, lse = torch.empty(40, 32, 128, device="cuda"), torch.empty(40, 32, device="cuda")
+        ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(5000, [100] * 40, 32, 8, 128))
+        run = lambda: ta.tree_attn_decode_bifurcated_ex(d["q"], d["k_prefix"], d["v_prefix"], 5000,  # noqa: E731
+                                                        d["k_suffix"], d["v_suffix"], [100] * 40, 32, 8, 128,
+                                                        sp.scale, out, lse, None, ws)
+    else:
+        sp = synth.AnchorSpec("p", 4096, 1024, 32, 8, 128, seed=48)
+        inp = synth.make_anchor_inputs(sp)
+        q, k, v = (device_tensor(inp[n], "bf16") for n in ("q", "k", "v"))
+        out, lse = torch.empty(4096, 32, 128, device="cuda"), torch.empty(4096, 32, device="cuda")
+        ws = new_workspace(256)
+        run = lambda: ta.tree_attn_anchor_prefill(q, k, v, 4096, 1024, 32, 8, 128, sp.scale, out, lse,  # noqa: E731
+                                                  None, ws)
+    run()  # warm (first-call set-up outside the spans)
+    ta.tree_attn_profile_events(inner[0], inner[1])
+    outer[0].record()
+    run()
+    outer[1].record()
+    ta.tree_attn_profile_events()
+    torch.cuda.synchronize()
+    assert ta.tree_attn_check(ws) == ta.TA_OK
+    whole = outer[0].elapsed_time(outer[1])
+    kernel = inner[0].elapsed_time(inner[1])
+    assert 0.0 < kernel <= whole
+    assert outer[0].elapsed_time(inner[0]) >= 0.0 and inner[1].elapsed_time(outer[1]) >= 0.0
+    # hook off: the next call leaves the events where they were
+    stamp = inner[1].elapsed_time(outer[1])
+    run()
+    torch.cuda.synchronize()
+    assert inner[1].elapsed_time(outer[1]) == stamp
