@@ -366,10 +366,12 @@ class DecodeRun:
     launches_per_step = 1
     metric, unit, bound = METRIC, UNIT, "hbm"
 
-    def __init__(self, spec, torch, ta, keep_inputs=False):
+    def __init__(self, spec, torch, ta, keep_inputs=False, decode_path=0):
         self.spec, self.torch, self.ta = spec, torch, ta
         B, Hq, Hkv, D = spec.batch, spec.n_q_heads, spec.n_kv_heads, spec.head_dim
         self.seqlens = [int(s) for s in spec.seqlens]
+        # ta_options.prefix_path for plain decode: 0 automatic, 1 tensor cores, 2 split kernel
+        self.opts = ta.make_options(prefix_path=decode_path) if decode_path else None
         inp = synth.make_decode_inputs(spec)
         self.host = {n: to_device_bf16(torch, inp[n]) for n in ("q", "k", "v")}
         self.inputs = inp if keep_inputs else None
@@ -377,20 +379,21 @@ class DecodeRun:
         self.dev = {n: t.cuda() for n, t in self.host.items()}
         self.out = torch.empty(B, Hq, D, device="cuda")
         self.lse = torch.empty(B, Hq, device="cuda")
-        self.ws = torch.empty(ta.tree_attn_workspace_size(self.seqlens, Hq, Hkv, D), dtype=torch.uint8, device="cuda")
+        self.ws = torch.empty(ta.tree_attn_workspace_size(self.seqlens, Hq, Hkv, D, "bf16", self.opts),
+                              dtype=torch.uint8, device="cuda")
         ta.tree_attn_workspace_init(self.ws)
         self.kv_bytes = spec.kv_bytes
         self.tokens = spec.tokens
         self.flops = 4 * D * Hq * sum(self.seqlens)
         self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv},{'ShortTiles' if sum(self.seqlens) < 1024 * len(self.seqlens) else 'LongTiles'}>"
-        if D == 128 and Hq // Hkv == 8:  # bf16 decode with G = 8 runs on the tensor cores
+        if D == 128 and ((Hq // Hkv == 8 and decode_path != 2) or decode_path == 1):  # tensor-core decode
             self.launches_per_step = 2 * ((B + 127) // 128)
-            self.kernel = "bif_prefix_kernel (decode, 8 rows per KV head)"
+            self.kernel = f"bif_prefix_kernel (decode, {Hq // Hkv} rows per KV head)"
 
     def step(self, stream):
         sp = self.spec
         self.ta.tree_attn_decode_ex("bf16", self.dev["q"], self.dev["k"], self.dev["v"], self.seqlens, sp.n_q_heads,
-                                    sp.n_kv_heads, sp.head_dim, sp.scale, self.out, self.lse, None, self.ws,
+                                    sp.n_kv_heads, sp.head_dim, sp.scale, self.out, self.lse, self.opts, self.ws,
                                     stream=stream)
 
 
@@ -557,7 +560,7 @@ class AnchorRun:
                                          stream=stream)
 
 
-def make_run(spec, torch, ta, keep_inputs=False):
+def make_run(spec, torch, ta, keep_inputs=False, decode_path=0):
     if isinstance(spec, synth.BifurcatedSpec):
         return BifurcatedRun(spec, torch, ta)
     if isinstance(spec, synth.AnchorSpec):
@@ -568,7 +571,7 @@ def make_run(spec, torch, ta, keep_inputs=False):
         return MultiRun(spec, torch, ta, keep_inputs)
     if spec.page_size > 0:
         return PagedRun(spec, torch, ta, keep_inputs)
-    return DecodeRun(spec, torch, ta, keep_inputs)
+    return DecodeRun(spec, torch, ta, keep_inputs, decode_path)
 
 
 def run_gpu(args, spec) -> None:
@@ -587,7 +590,7 @@ def run_gpu(args, spec) -> None:
 
     want_cpu = world == 1 and not args.no_cpu_baseline and isinstance(spec, synth.DecodeSpec) and \
         spec.n_queries == 1 and spec.page_size == 0
-    run = make_run(spec, torch, ta, keep_inputs=want_cpu)
+    run = make_run(spec, torch, ta, keep_inputs=want_cpu, decode_path=DECODE_PATHS[args.decode_path])
     stream = torch.cuda.current_stream()
     small = spec.kv_bytes <= 2 * 126e6
     flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda") if small else None
@@ -687,6 +690,8 @@ def run_gpu(args, spec) -> None:
         extra["cpu_baseline"] = cpu_baseline(spec, run.inputs)
     rec = make_record(metric=run.metric, unit=run.unit, value=value, n_gpus=world, steps=args.steps,
                       warmup=args.warmup, ms_per_step=ms_per_step, spec=spec, dtype="bf16", extra=extra)
+    if args.decode_path != "auto":
+        rec["config"]["decode_path"] = args.decode_path
     if rank == 0:
         print(json.dumps(rec), flush=True)
     if world > 1:
@@ -695,9 +700,13 @@ def run_gpu(args, spec) -> None:
         dist.destroy_process_group()
 
 
+DECODE_PATHS = {"auto": 0, "tensor": 1, "split": 2}
+
+
 def all_workloads():
-    return {**synth.decode_configs(), **synth.capture_configs(), **synth.bifurcated_configs(),
-            **synth.multi_query_configs(), **synth.paged_configs(), **synth.anchor_configs()}
+    return {**synth.decode_configs(), **synth.gqa8_configs(), **synth.capture_configs(),
+            **synth.bifurcated_configs(), **synth.multi_query_configs(), **synth.paged_configs(),
+            **synth.anchor_configs()}
 
 
 def main(argv=None):
@@ -709,6 +718,8 @@ def main(argv=None):
     workloads = all_workloads()
     ap.add_argument("--workload", default="long_1m", choices=sorted(workloads))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-path", default="auto", choices=sorted(DECODE_PATHS),
+                    help="plain decode workloads: the library's choice, or force the tensor-core or split kernel")
     args = ap.parse_args(argv)
     spec = workloads[args.workload]
     if args.impl == "reference":

@@ -351,6 +351,8 @@ bool decode_on_tensor_cores(const DecodeArgs& a, const ta_options* opts) {
   return path == 1 || (path == 0 && a.Hq / a.Hkv == 8);
 }
 
+ta_status decode_workspace_bytes(const DecodeArgs& a, const ta_options* opts, const KernelInfo& ki, size_t* bytes);
+
 // Decode through the several-query form (defined with it, below); with bytes_only it only
 // reports the workspace size.
 ta_status decode_tc(const DecodeArgs& a, const ta_options* opts, void* ws, size_t ws_bytes, cudaStream_t st,
@@ -551,6 +553,24 @@ ta_status multi_run(const DecodeArgs& a, int n_queries, const ta_options* opts, 
                             a.Hq, err, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
+  return TA_OK;
+}
+
+// Workspace of a decode call: the split plan's, or, when the call goes to the tensor cores, the
+// larger of that and the tensor-core plan's (a paged call whose page pool is too large for the
+// tensor maps falls back to the split plan, so either must fit).
+ta_status decode_workspace_bytes(const DecodeArgs& a, const ta_options* opts, const KernelInfo& ki, size_t* bytes) {
+  Plan plan;
+  ta_status s = plan_for(a, opts, ki, &plan);
+  if (s != TA_OK) return s;
+  size_t n = kHeaderBytes + plan.body_bytes;
+  if (a.batch > 0 && decode_on_tensor_cores(a, opts)) {
+    size_t tc = 0;
+    s = decode_tc(a, opts, nullptr, 0, nullptr, &tc);
+    if (s != TA_OK) return s;
+    n = std::max(n, tc);
+  }
+  *bytes = n;
   return TA_OK;
 }
 
@@ -909,14 +929,9 @@ ta_status tree_attn_workspace_size(const int64_t* seqlens, int32_t batch, int32_
   DecodeArgs a{dtype, nullptr, nullptr, nullptr, seqlens, nullptr, batch, n_q_heads, n_kv_heads, head_dim,
                1.0f, nullptr, nullptr};
   KernelInfo ki;
-  Plan plan;
   ta_status s = validate(a, opts, false, &ki);
   if (s != TA_OK) return s;
-  if (batch > 0 && decode_on_tensor_cores(a, opts)) return decode_tc(a, opts, nullptr, 0, nullptr, bytes);
-  s = plan_for(a, opts, ki, &plan);
-  if (s != TA_OK) return s;
-  *bytes = kHeaderBytes + plan.body_bytes;
-  return TA_OK;
+  return decode_workspace_bytes(a, opts, ki, bytes);
 }
 
 ta_status tree_attn_workspace_init(void* ws, size_t ws_bytes, void* stream) {
@@ -949,12 +964,7 @@ ta_status decode_alloc(const DecodeArgs& a, cudaStream_t st) {
   if (s != TA_OK) return s;
   if (a.batch == 0) return TA_OK;
   size_t bytes = 0;
-  if (decode_on_tensor_cores(a, nullptr)) {
-    s = decode_tc(a, nullptr, nullptr, 0, st, &bytes);
-  } else {
-    s = plan_for(a, nullptr, ki, &plan);
-    bytes = kHeaderBytes + plan.body_bytes;
-  }
+  s = decode_workspace_bytes(a, nullptr, ki, &bytes);
   if (s != TA_OK) return s;
   PlainCtx ctx{a};
   return with_temp_workspace(bytes, st, &plain_run, &ctx);
@@ -1157,6 +1167,13 @@ ta_status paged_run(const PagedArgs& pa, const ta_options* opts, void* ws, size_
   if (s != TA_OK) return s;
   if (a.batch == 0) return TA_OK;
   if (!ws || !aligned(ws, kAlign)) return TA_ERR_WORKSPACE;
+  if (decode_on_tensor_cores(a, opts)) {  // G = 8 (or forced): the paged tensor-core form, one query token
+    if (!pc.table || (reinterpret_cast<uintptr_t>(pc.table) & 3) != 0) return TA_ERR_INVALID_ARG;
+    MultiPlan mp;
+    s = multi_plan(a, 1, opts, &mp, &pc);
+    if (s != TA_OK) return s;
+    return multi_run(a, 1, opts, mp, ws, ws_bytes, st, &pc);
+  }
   Plan plan;
   s = plan_for(a, opts, ki, &plan);
   if (s != TA_OK) return s;
@@ -1198,11 +1215,10 @@ ta_status tree_attn_decode_paged(const void* q, const void* k_pages, const void*
   PagedCache pc;
   ta_status s = paged_validate(pa.a, pa.pc, page_size, nullptr, true, &ki, &pc);
   if (s != TA_OK || batch == 0) return s;
-  Plan plan;
-  s = plan_for(pa.a, nullptr, ki, &plan);
+  size_t bytes = 0;
+  s = decode_workspace_bytes(pa.a, nullptr, ki, &bytes);
   if (s != TA_OK) return s;
-  return with_temp_workspace(kHeaderBytes + plan.body_bytes, static_cast<cudaStream_t>(stream), &paged_alloc_run,
-                             &pa);
+  return with_temp_workspace(bytes, static_cast<cudaStream_t>(stream), &paged_alloc_run, &pa);
 }
 
 // ------------------------------------------------------------------------------------------

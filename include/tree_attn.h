@@ -285,7 +285,9 @@ ta_status tree_attn_noalloc_check(void* stream);
  *                     block_table[b * block_table_stride + i]; stride >= ceil(max S_b / page_size)
  *   page_size         a power of two >= 16 (TA_ERR_INVALID_ARG otherwise)
  * q, out, lse, seqlens, workspace (tree_attn_workspace_size applies unchanged) and the other
- * rules as tree_attn_decode_ex.  Every entry a sequence uses is checked against num_pages on
+ * rules as tree_attn_decode_ex; bf16 calls with head_dim 128 and G = 8 run on the paged
+ * tensor-core form (as tree_attn_decode_multi_paged_ex with one query token; prefix_path
+ * selects the path).  Every entry a sequence uses is checked against num_pages on
  * the device before anything is read through it: an entry outside [0, num_pages) makes
  * tree_attn_check report TA_ERR_BAD_PAGE and the affected outputs NaN.
  */

@@ -196,6 +196,12 @@ def decode_configs() -> Dict[str, DecodeSpec]:
     }
 
 
+def gqa8_configs() -> Dict[str, DecodeSpec]:
+    """Decode with 8 query heads per KV head (Llama-3-70B-shaped: 64 query heads, 8 KV heads,
+    head_dim 128) over long_1m's recipe: 1,048,576 tokens, bf16, 0.1% of keys scaled x4."""
+    return {"long_1m_g8": DecodeSpec("long_1m_g8", [1_048_576], 64, 8, 128, seed=12, spike_frac=0.001)}
+
+
 def multi_query_configs() -> Dict[str, DecodeSpec]:
     """Several query tokens per sequence (speculative decode verifying draft tokens): the
     32K x 8 batch of llama3_8b_gqa with 2 and with 4 query tokens per sequence."""

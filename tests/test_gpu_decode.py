@@ -194,7 +194,7 @@ def _full_size(name, workers=0):
     of one (sequence, KV head) computed side by side on the host cores."""
     from gpu_util import oracle_parallel
 
-    sp = synth.decode_configs()[name]
+    sp = {**synth.decode_configs(), **synth.gqa8_configs()}[name]
     inp = synth.make_decode_inputs(sp)
     out, lse = decode_gpu(inp, sp)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
@@ -214,3 +214,8 @@ def test_config_extreme_5m_all_rows():
 
 def test_config_extreme_ragged_all_rows():
     _full_size("extreme_ragged", workers=4)
+
+
+def test_config_long_1m_g8_all_rows():
+    """64 query heads over 8 KV heads at 1M tokens: the tensor-core decode path."""
+    _full_size("long_1m_g8")

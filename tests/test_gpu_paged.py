@@ -238,3 +238,30 @@ def test_multi_query_paged_bad_entry():
                                        out, lse, opts, ws)
     assert ta.tree_attn_check(ws) == ta.TA_ERR_BAD_PAGE
     assert np.isnan(out[0].cpu().numpy()).all()
+
+
+@pytest.mark.parametrize("path", [0, 2])
+@pytest.mark.parametrize("ps", [16, 64, 256])
+def test_paged_g8_decode(ps, path):
+    """G = 8 bf16 decode over pages runs on the paged tensor-core form by default (one query token)
+    and on the split kernel with prefix_path 2; both against the oracle, unused page rows NaN."""
+    import exact_long_context_split_b200 as ta
+
+    sp, inp, table, n_pages, kp, vp = paged_case([1, 0, 300, 5000, 129], 16, 2, 128, "bf16", ps, seed=11)
+    opts = ta.make_options(prefix_path=path) if path else None
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, ps, opts)
+    compare(out, lse, *oracle_paged(sp, inp, table, kp, vp, ps))
+
+
+def test_paged_g8_bad_entry_and_allocating_entry():
+    """On the tensor-core route a bad block-table entry is reported (TA_ERR_BAD_PAGE, NaN outputs)
+    and the allocating entry point sizes its workspace for that route."""
+    import exact_long_context_split_b200 as ta
+
+    sp, inp, table, n_pages, kp, vp = paged_case([700, 33], 64, 8, 128, "bf16", 16, seed=12, spare=0)
+    bad = table.copy()
+    bad[0, 7] = n_pages
+    out, lse = paged_gpu(sp, inp, bad, n_pages, kp, vp, 16, expect=ta.TA_ERR_BAD_PAGE)
+    assert np.isnan(out).all() and np.isnan(lse).all()
+    out, lse = paged_gpu(sp, inp, table, n_pages, kp, vp, 16, entry="alloc")
+    compare(out, lse, *oracle_paged(sp, inp, table, kp, vp, 16))
