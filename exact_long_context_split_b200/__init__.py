@@ -64,7 +64,8 @@ class ta_options(ctypes.Structure):
         ("debug_skip_tile", ctypes.c_int32),
         ("prefix_path", ctypes.c_int32),
         ("split_tiles", ctypes.c_int32),
-        ("reserved", ctypes.c_int32 * 3),
+        ("debug_skip_stage", ctypes.c_int32),
+        ("reserved", ctypes.c_int32 * 2),
     ]
 
 
@@ -75,8 +76,10 @@ TILES_AUTO, TILES_LONG, TILES_SHORT = 0, 1, 2
 
 
 def make_options(num_ctas: int = 0, wait_limit_us: int = 0, debug_skip_tile: int = -1,
-                 prefix_path: int = PREFIX_AUTO, split_tiles: int = TILES_AUTO) -> ta_options:
-    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, prefix_path, split_tiles, (ctypes.c_int32 * 3)())
+                 prefix_path: int = PREFIX_AUTO, split_tiles: int = TILES_AUTO,
+                 debug_skip_stage: int = 0) -> ta_options:
+    return ta_options(num_ctas, wait_limit_us, debug_skip_tile, prefix_path, split_tiles, debug_skip_stage,
+                      (ctypes.c_int32 * 2)())
 
 
 _lib = None

@@ -364,6 +364,10 @@ __global__ void __launch_bounds__(kBifThreads, 1)
   const uint32_t raw = smem_addr(bif_smem_raw);
   BifSmem& sm = *reinterpret_cast<BifSmem*>(bif_smem_raw + (((raw + 1023u) & ~1023u) - raw));
 
+  // A kernel launched after this one with programmatic dependent launch (the short-unit suffix
+  // pass) may start on the SMs this grid leaves free; it waits for this grid's completion before
+  // it reads anything this kernel writes.
+  asm volatile("griddepcontrol.launch_dependents;");
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;

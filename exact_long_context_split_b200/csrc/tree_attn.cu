@@ -191,10 +191,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 ta_status check_opts(const ta_options* o) {
   if (!o) return TA_OK;
-  if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1) return TA_ERR_INVALID_ARG;
+  if (o->num_ctas < 0 || o->wait_limit_us < 0 || o->debug_skip_tile < -1 || o->debug_skip_stage < 0)
+    return TA_ERR_INVALID_ARG;
   if (o->prefix_path < 0 || o->prefix_path > 2) return TA_ERR_INVALID_ARG;
   if (o->split_tiles < 0 || o->split_tiles > 3) return TA_ERR_INVALID_ARG;
-  for (int i = 0; i < 3; ++i)
+  for (int i = 0; i < 2; ++i)
     if (o->reserved[i] != 0) return TA_ERR_INVALID_ARG;
   return TA_OK;
 }
@@ -670,6 +671,7 @@ struct BifPlan {
   int mtiles = 0, chunks = 0, rows_per_head = 0;
   size_t part_off = 0;
   bool short_suffix = false;  // suffix pass on the short-unit kernel (tensor-core prefix pass only)
+  int sms = 0;
 };
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
@@ -773,6 +775,7 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
     s = bif_tc_setup(&sms);
     if (s != TA_OK) return s;
     bp->tc = true;
+    bp->sms = sms;
     bp->rows_per_head = a.N * (a.Hq / a.Hkv);
     bp->mtiles = (bp->rows_per_head + kBifMT * kBifRows - 1) / (kBifMT * kBifRows);  // CTAs per (chunk, head)
     const int64_t tiles = (a.P + kBifKeys - 1) / kBifKeys;
@@ -793,8 +796,10 @@ ta_status bif_plan(const BifArgs& a, const ta_options* opts, const KernelInfo& k
   return TA_OK;
 }
 
-// The suffix pass on the short-unit kernel: one launch per 128 samples.
-ta_status launch_short(const BifArgs& a, const PrefixFold& pf, int* err, cudaStream_t st) {
+// The suffix pass on the short-unit kernel: one launch per 128 samples, the first of them
+// allowed to start while the prefix pass (the stream's previous kernel) still runs.
+ta_status launch_short(const BifArgs& a, const ta_options* opts, int sms, const PrefixFold& pf, int* err,
+                       cudaStream_t st) {
   const int G = a.Hq / a.Hkv;
   int64_t off = 0;
   for (int b0 = 0; b0 < a.N; b0 += kShortMaxSeq) {
@@ -813,13 +818,16 @@ ta_status launch_short(const BifArgs& a, const PrefixFold& pf, int* err, cudaStr
     sp.pre_stride = pf.stride;
     sp.n_kv_heads = a.Hkv;
     sp.n_q_heads = a.Hq;
+    sp.n_seq = nb;
     sp.scale_log2 = static_cast<float>(static_cast<double>(a.scale) * 1.4426950408889634073599246810019);
+    sp.wait_limit_ns = 1000LL * ((opts && opts->wait_limit_us > 0) ? opts->wait_limit_us : kDefaultWaitUs);
+    sp.debug_skip_stage1 = (opts && b0 == 0) ? opts->debug_skip_stage : 0;
     for (int i = 0; i < nb; ++i) {
       sp.kv_off[i] = off;
       sp.seq_len[i] = a.suffix_lens[b0 + i];
       off += a.suffix_lens[b0 + i] * a.Hkv * a.D;
     }
-    const cudaError_t e = launch_short_decode(G, a.Hkv, nb, sp, st);
+    const cudaError_t e = launch_short_decode(G, sp, sms, opts ? opts->num_ctas : 0, b0 == 0, st);
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return TA_OK;
@@ -871,7 +879,7 @@ ta_status bif_run(const BifArgs& a, const ta_options* opts, const BifPlan& bp, v
       pf.rows = bp.rows_per_head;
       pf.stride = kBifPartRow;
       if (bp.short_suffix)
-        s = launch_short(a, pf, err, st);
+        s = launch_short(a, opts, bp.sms, pf, err, st);
       else
         s = launch_plan(bp.suffix, bp.ki_suffix, a.q, a.ks, a.vs, a.out, a.lse, a.Hq, a.Hkv, a.D, a.scale, TA_BF16,
                         opts, base + bp.suffix_off, err, st, 1, 0, nullptr, &pf);

@@ -97,7 +97,9 @@ typedef struct {
                               runs on the short-unit kernel (one CTA per sample and KV head) when
                               head_dim is 128, there are at least as many (sample, KV head) units as
                               SMs and no suffix exceeds 2048 tokens, or always with 3 */
-  int32_t reserved[3];     /* must be 0 */
+  int32_t debug_skip_stage; /* 0: off.  Test hook of the short-unit suffix kernel: s > 0 makes its
+                              CTA 0 never load its key stage s - 1, so that stage's wait runs out */
+  int32_t reserved[2];     /* must be 0 */
 } ta_options;
 
 /*

@@ -77,8 +77,9 @@ def test_decode_ex_rejects(kwargs, status):
 
 def test_reserved_options_must_be_zero():
     o = ta.make_options()
-    o.reserved[2] = 1
+    o.reserved[1] = 1
     assert call_ex(opts=o) == ta.TA_ERR_INVALID_ARG
+    assert call_ex(opts=ta.make_options(debug_skip_stage=-1)) == ta.TA_ERR_INVALID_ARG
 
 
 def test_bad_dtype_rejected():

@@ -9,7 +9,7 @@ from gpu_util import compare, device_tensor, empty_outputs, new_workspace
 pytestmark = pytest.mark.gpu
 
 
-def bif_gpu(inp, sp, entry="ex", prefix_path=0, split_tiles=0):
+def bif_gpu(inp, sp, entry="ex", prefix_path=0, split_tiles=0, num_ctas=0):
     import torch
 
     import exact_long_context_split_b200 as ta
@@ -21,7 +21,7 @@ def bif_gpu(inp, sp, entry="ex", prefix_path=0, split_tiles=0):
     out, lse = empty_outputs(N, Hq, D)
     lens = [int(s) for s in sp.suffix_lens]
     if entry == "ex":
-        opts = ta.make_options(prefix_path=prefix_path, split_tiles=split_tiles)
+        opts = ta.make_options(num_ctas=num_ctas, prefix_path=prefix_path, split_tiles=split_tiles)
         ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(P, lens, Hq, Hkv, D, opts))
         ta.tree_attn_decode_bifurcated_ex(q, kp, vp, P, ks, vs, lens, Hq, Hkv, D, sp.scale, out, lse, opts, ws)
         assert ta.tree_attn_check(ws) == ta.TA_OK
@@ -96,6 +96,41 @@ def test_short_unit_suffix_pass(prefix_len, suffix_lens, Hq, Hkv, D):
     compare(out, lse, *oracle_bif(inp, sp))
     again = bif_gpu(inp, sp, "ex", prefix_path=1, split_tiles=3)
     assert np.array_equal(out.view(np.uint32), again[0].view(np.uint32))
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 7, 40])
+def test_short_unit_suffix_grid_sizes(num_ctas):
+    """Fewer persistent CTAs than units: each CTA streams several ragged units through its stage
+    ring (wrapping it many times, units with 0, 1 and partial stages), against the oracle."""
+    sp = synth.BifurcatedSpec("case", 700, [0, 1, 31, 32, 33, 255, 256, 257, 600, 5] * 3, 32, 8, 128, seed=26)
+    inp = synth.make_bifurcated_inputs(sp)
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path=1, split_tiles=3, num_ctas=num_ctas)
+    compare(out, lse, *oracle_bif(inp, sp))
+
+
+def test_short_unit_suffix_stage_never_loaded():
+    """The suffix kernel's bounded waits: with a stage of CTA 0 never loaded, the call reports
+    TA_ERR_TIMEOUT, CTA 0's first unit (sample 0, KV head 0) comes out NaN, and the next call on
+    the same stream is correct."""
+    import torch
+
+    import exact_long_context_split_b200 as ta
+
+    sp = synth.BifurcatedSpec("case", 1000, [300, 40, 7, 128], 32, 8, 128, seed=27)
+    inp = synth.make_bifurcated_inputs(sp)
+    q = device_tensor(inp["q"], "bf16")
+    kp, vp = device_tensor(inp["k_prefix"], "bf16"), device_tensor(inp["v_prefix"], "bf16")
+    ks, vs = device_tensor(inp["k_suffix"], "bf16"), device_tensor(inp["v_suffix"], "bf16")
+    lens = [int(s) for s in sp.suffix_lens]
+    for skip in (1, 3, 9):
+        out, lse = torch.zeros(4, 32, 128, device="cuda"), torch.zeros(4, 32, device="cuda")
+        opts = ta.make_options(wait_limit_us=20000, prefix_path=1, split_tiles=3, debug_skip_stage=skip)
+        ws = new_workspace(ta.tree_attn_bifurcated_workspace_size(1000, lens, 32, 8, 128, opts))
+        ta.tree_attn_decode_bifurcated_ex(q, kp, vp, 1000, ks, vs, lens, 32, 8, 128, sp.scale, out, lse, opts, ws)
+        assert ta.tree_attn_check(ws) == ta.TA_ERR_TIMEOUT
+        assert torch.isnan(out[0, :4]).all() and torch.isnan(lse[0, :4]).all()
+    out, lse = bif_gpu(inp, sp, "ex", prefix_path=1, split_tiles=3)
+    compare(out, lse, *oracle_bif(inp, sp))
 
 
 def test_tensor_core_prefix_is_deterministic():
