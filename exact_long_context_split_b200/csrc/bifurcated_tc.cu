@@ -27,9 +27,19 @@ cudaError_t launch_merge_chunks(const float* part, int n_chunks, int n_kv_heads,
                                 float* out, float* lse, int batch, int n_q_heads, const int* err, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(batch) * n_queries * n_q_heads * (kBifD / 4);  // one thread per 4 columns
   if (n == 0) return cudaSuccess;
-  merge_chunks_kernel<<<static_cast<unsigned>((n + 127) / 128), 128, 0, st>>>(
-      part, n_chunks, n_kv_heads, rows_per_head, n_queries, out, lse, batch, n_q_heads, err);
-  return cudaGetLastError();
+  // Launched as a dependent of the tensor-core pass before it (programmatic dependent launch):
+  // its blocks are scheduled while that kernel's last CTAs run and wait for its completion.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((n + 127) / 128));
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_chunks_kernel, part, n_chunks, n_kv_heads, rows_per_head, n_queries, out,
+                            lse, batch, n_q_heads, err);
 }
 
 }  // namespace ta

@@ -827,6 +827,9 @@ __global__ void __launch_bounds__(128) merge_chunks_kernel(const float* __restri
                                                            float* __restrict__ out, float* __restrict__ lse,
                                                            int batch, int n_q_heads, const int* __restrict__ err) {
   constexpr int Q = kBifD / 4;
+  // The partials are those of the kernel launched before this one: wait for its completion
+  // (immediate when this launch was not a programmatic dependent).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total = static_cast<int64_t>(batch) * n_queries * n_q_heads * Q;
   if (i >= total) return;
