@@ -17,8 +17,8 @@ step of the workload (all rows), threaded over (sequence, query head) rows.
 Other workloads (--workload): the decode configurations, several query tokens per
 sequence, paged caches, the shared-prefix (bifurcated) step and context encoding with
 anchor blocks.  Each line's roofline is that of the step's main kernel, timed with CUDA
-events that the library records around its launches (tree_attn_profile_events) in a second
-set of K steps; the step time comes from steps without those events.
+events that the library records around its launches (tree_attn_profile_events) in K steps
+interleaved with the K timed steps, which carry no such events.
 """
 from __future__ import annotations
 
@@ -616,19 +616,19 @@ def run_gpu(args, spec) -> None:
         clocks.start()
         # The step time comes from steps with no library events inside them (an event between
         # two of the step's launches would serialise a launch meant to overlap its predecessor);
-        # the main kernel's time from a second set of steps with the library's events around it.
+        # the main kernel's time from steps interleaved with them, with the library's events
+        # around that kernel.
         for i in range(args.steps):
             if flush is not None:
                 flush.fill_(i & 0xFF)  # L2 flush outside the step's events
             starts[i].record(stream)
             run.step(stream)
             ends[i].record(stream)
-        for i in range(args.steps):
             if flush is not None:
-                flush.fill_(i & 0xFF)
+                flush.fill_((i + 128) & 0xFF)
             ta.tree_attn_profile_events(kstarts[i], kends[i])
             run.step(stream)
-        ta.tree_attn_profile_events()
+            ta.tree_attn_profile_events()
         torch.cuda.synchronize()
         clocks.stop()
         barrier(world)
