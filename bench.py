@@ -44,8 +44,13 @@ UNIT = "GB/s"
 ANCHOR_METRIC = "context-encoding attention TFLOP/s (anchor-block mask, exact); µs/step, tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["exact_long_context_split_b200/csrc/split_kv.cuh", "exact_long_context_split_b200/csrc/ptx.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kv_traffic.json")
+# DRAM traffic per launch from committed ncu captures, per family of main kernel: the capture
+# file and the sources it was taken from (a capture counts only while they are unchanged).
+_CSRC = "exact_long_context_split_b200/csrc/"
+TRAFFIC = {
+    "split": ("split_kv_traffic.json", [_CSRC + "split_kv.cuh", _CSRC + "ptx.cuh"]),
+    "tc_decode": ("bif_prefix_decode_traffic.json", [_CSRC + "bifurcated_tc.cuh", _CSRC + "ptx.cuh"]),
+}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -77,9 +82,9 @@ def barrier(world: int) -> None:
         dist.barrier()
 
 
-def kernel_hash() -> str:
+def kernel_hash(sources) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -97,16 +102,20 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def traffic_per_launch(spec) -> object:
-    """DRAM bytes (read + write) of one launch from the committed ncu capture: the mean of the
-    captured launches for the captured workload, reads scaled by K/V bytes for another one.
-    None when the kernel sources changed since the counters were taken."""
+def traffic_per_launch(spec, family) -> object:
+    """DRAM bytes (read + write) of one launch of the family's main kernel from its committed ncu
+    capture: the mean of the captured launches for the captured workload, reads scaled by K/V
+    bytes for another one.  None without a capture, or when the kernel's sources changed since
+    the counters were taken."""
+    if family not in TRAFFIC:
+        return None
+    name, sources = TRAFFIC[family]
     try:
-        with open(TRAFFIC_FILE) as fh:
+        with open(os.path.join(ROOT, "profiles", name)) as fh:
             d = json.load(fh)
     except Exception:
         return None
-    if d.get("kernel_hash") != kernel_hash():
+    if d.get("kernel_hash") != kernel_hash(sources):
         return None
     rd = statistics.mean(d["dram_bytes_read"])
     wr = statistics.mean(d["dram_bytes_write"])
@@ -387,7 +396,9 @@ class DecodeRun:
         self.tokens = spec.tokens
         self.flops = 4 * D * Hq * sum(self.seqlens)
         self.kernel = f"split_kv_decode_kernel<bf16,{D},{Hq // Hkv},{'ShortTiles' if sum(self.seqlens) < 1024 * len(self.seqlens) else 'LongTiles'}>"
+        self.family = "split"
         if D == 128 and ((Hq // Hkv == 8 and decode_path != 2) or decode_path == 1):  # tensor-core decode
+            self.family = "tc_decode"
             self.launches_per_step = 2 * ((B + 127) // 128)
             self.kernel = f"bif_prefix_kernel (decode, {Hq // Hkv} rows per KV head)"
 
@@ -678,7 +689,7 @@ def run_gpu(args, spec) -> None:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_kind": peak_kind + " copy bandwidth", "bytes_per_launch": run.kv_bytes}
     roof.update({"kernel": run.kernel, "kernel_us": kernel_ms * 1e3,
-                 "traffic": traffic_per_launch(spec) if type(run) is DecodeRun else None})
+                 "traffic": traffic_per_launch(spec, run.family) if type(run) is DecodeRun else None})
     extra = {
         "us_per_step": ms_per_step * 1e3,
         "kv_tokens_per_s": world * run.tokens * args.steps / elapsed_s,
