@@ -704,7 +704,7 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
         if (tid == 0) sm.is_last = (atomicAdd(&p.tickets[unit], 1) == n_parts - 1);
         named_barrier(1, C::NCT);
         if (sm.is_last) {
-          // 3) last CTA of the unit: fixed pairwise tree over the unit's partials
+          // 3) last CTA of the unit: a tree over the unit's partials fixed by their count
           __threadfence();
           const float* base = p.part + static_cast<int64_t>(i_first + unit) * C::SLOT;
           const int n = n_parts;
@@ -730,8 +730,10 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
               const int col = tid + k * C::NCT;
               if (col < G * D) {
                 const int g = col / D, d = col % D;
-                // Leaves in batches of 16: the batch's loads are in flight together, then
-                // enter the pairwise sum in order.
+                // Leaves in batches of 16: the batch's loads are in flight together; each batch
+                // is summed by a fixed balanced tree (in registers) and its sum enters the
+                // pairwise sum in order, one push per batch (the pairwise state is indexed at run
+                // time and lives in local memory).
                 constexpr int LB = 16;
                 for (int cb = 0; cb < nb; cb += LB) {
                   float ov[LB], lv[LB];
@@ -744,11 +746,12 @@ __global__ void __launch_bounds__(SplitCfg<T, D, G, V>::THREADS, 1)
                   }
 #pragma unroll
                   for (int u = 0; u < LB; ++u) {
-                    if (cb + u < nb) {
-                      acc[k].push(sm.mw[cb + u][g] * ov[u]);
-                      if (d == 0) accl[k].push(sm.mw[cb + u][g] * lv[u]);
-                    }
+                    const float wgt = (cb + u < nb) ? sm.mw[cb + u][g] : 0.f;
+                    ov[u] *= wgt;
+                    lv[u] *= wgt;
                   }
+                  acc[k].push(tree_sum<LB>(ov));
+                  if (d == 0) accl[k].push(tree_sum<LB>(lv));
                 }
               }
             }
