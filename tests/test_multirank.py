@@ -96,6 +96,25 @@ def test_reference_arm_runs_full_steps_on_the_host():
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
 
 
+def test_traffic_capture_follows_its_kernel_family(monkeypatch):
+    """A committed DRAM-traffic capture is attached only to the kernel family it was taken on,
+    scaled by K/V bytes for another workload of that family, and dropped once its kernel's
+    sources differ from the ones it was taken from."""
+    import bench
+
+    specs = bench.all_workloads()
+    split = bench.traffic_per_launch(specs["long_1m"], "split")
+    tc = bench.traffic_per_launch(specs["long_1m_g8"], "tc_decode")
+    assert isinstance(split, int) and isinstance(tc, int)
+    kv = specs["long_1m"].kv_bytes
+    assert kv <= split <= 1.01 * kv and kv <= tc <= 1.01 * kv
+    quarter = bench.traffic_per_launch(specs["long_256k"], "split")
+    assert abs(quarter - split / 4) < 0.01 * split  # reads scale with the K/V bytes
+    assert bench.traffic_per_launch(specs["long_1m"], "paged") is None
+    monkeypatch.setattr(bench, "kernel_hash", lambda sources: "0" * 16)
+    assert bench.traffic_per_launch(specs["long_1m"], "split") is None
+
+
 def test_clock_sampler_edges_without_nvml():
     """Without NVML the sampler reports why, and the bench still gets a summary."""
     sys.path.insert(0, ROOT)
