@@ -297,24 +297,22 @@ __device__ __forceinline__ void bif_exp_chunk(const float (&x)[32], uint32_t col
   tmem_st16u(col, h);
 }
 
-// Pass 2 over a full tile: the next 32 scores load while the current ones are exponentiated.
-// P chunk q goes to columns [16 q, 16 q + 16), below every score column still to be read.
+// Pass 2 over a full tile, 32 scores at a time.  P chunk q goes to columns [16 q, 16 q + 16),
+// below every score column still to be read.  (Loading the next 32 scores while the current
+// ones are exponentiated held two 32-column buffers and spilled registers to local memory on
+// this path, where each spill is an L2 round trip beside 224 KB of shared memory; the
+// one-buffer loop does the same operations in the same order without spills, and measured
+// 0.5-1% faster on every mode.)
 __device__ __forceinline__ float bif_tile_exp(uint32_t s_col, float sc, float mn) {
   const float2 s2 = make_float2(sc, sc), nm = make_float2(-mn, -mn);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-  float a[32], b[32];
-  tmem_ld32(s_col, a);
-  tmem_wait_ld_regs(a);
-  tmem_ld32(s_col + 32, b);
-  bif_exp_chunk(a, s_col, s2, nm, acc);
-  tmem_wait_ld_regs(b);
-  tmem_ld32(s_col + 64, a);
-  bif_exp_chunk(b, s_col + 16, s2, nm, acc);
-  tmem_wait_ld_regs(a);
-  tmem_ld32(s_col + 96, b);
-  bif_exp_chunk(a, s_col + 32, s2, nm, acc);
-  tmem_wait_ld_regs(b);
-  bif_exp_chunk(b, s_col + 48, s2, nm, acc);
+  float a[32];
+#pragma unroll 1
+  for (int q = 0; q < 4; ++q) {
+    tmem_ld32(s_col + 32 * q, a);
+    tmem_wait_ld_regs(a);
+    bif_exp_chunk(a, s_col + 16 * q, s2, nm, acc);
+  }
   const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
   const float2 a4 = __fadd2_rn(a01, a23);
   return a4.x + a4.y;

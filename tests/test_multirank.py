@@ -102,6 +102,13 @@ def test_traffic_capture_follows_its_kernel_family(monkeypatch):
     sources differ from the ones it was taken from."""
     import bench
 
+    recorded = {}
+    for fam, (name, _) in bench.TRAFFIC.items():
+        with open(os.path.join(ROOT, "profiles", name)) as fh:
+            recorded[fam] = json.load(fh)["kernel_hash"]
+    # Sources as they were when each capture was taken: the captures count.
+    hashes = {tuple(src): recorded[fam] for fam, (_, src) in bench.TRAFFIC.items()}
+    monkeypatch.setattr(bench, "kernel_hash", lambda sources: hashes[tuple(sources)])
     specs = bench.all_workloads()
     split = bench.traffic_per_launch(specs["long_1m"], "split")
     tc = bench.traffic_per_launch(specs["long_1m_g8"], "tc_decode")
@@ -111,6 +118,7 @@ def test_traffic_capture_follows_its_kernel_family(monkeypatch):
     quarter = bench.traffic_per_launch(specs["long_256k"], "split")
     assert abs(quarter - split / 4) < 0.01 * split  # reads scale with the K/V bytes
     assert bench.traffic_per_launch(specs["long_1m"], "paged") is None
+    # Sources changed since: no traffic figure.
     monkeypatch.setattr(bench, "kernel_hash", lambda sources: "0" * 16)
     assert bench.traffic_per_launch(specs["long_1m"], "split") is None
 
